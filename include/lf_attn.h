@@ -1,0 +1,142 @@
+/*
+ * lf_attn.h -- C ABI of liblfattn: Longformer sparse self-attention, forward,
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Operation (the "Longformer" note, eightmm.github.io/papers/architectures/
+ * longformer, sections "Sliding-Window Attention", "Global Attention" and
+ * "Mask View"; dilation as in the Longformer wiki, ciallo.wiki, section
+ * 2.2.3):
+ *
+ *   y[b,h,i] = sum_{j in N(i)} softmax_j( scale * q[b,h,i] . k[b,h,j] ) v[b,h,j]
+ *
+ *   N(i) = ( {i + dil[h]*t : |t| <= r} clipped to [0,T)  U  G_b ) \ padded keys
+ *          for i not in G_b;
+ *   N(i) = all non-padded keys, for i in G_b.
+ *
+ * G_b is the set of in-range entries of global_idx[b, :] (duplicates
+ * collapse; a global key inside the window is counted once).  A padded
+ * position is never a key; if it is also global it is still a global query.
+ * Rows whose key set is empty produce 0.  Every output row is written,
+ * padded query rows included.
+ *
+ * Conventions for every entry point:
+ *   - Tensors q, k, v, out are contiguous [B, H, T, d], row-major (d
+ *     innermost), all of the dtype given by `dtype`; they must be 16-byte
+ *     aligned.
+ *   - "device" pointers are CUDA device (or managed) memory of the current
+ *     device; "host" pointers are ordinary CPU memory.
+ *   - The caller owns every pointer; the library keeps none after return.
+ *     It owns one workspace per device (grown on demand with cudaMalloc,
+ *     freed by lf_attn_release).  Calls that use the same device share that
+ *     workspace, so calls on different streams of one device must not
+ *     overlap in time.  The first call that needs a larger workspace must
+ *     not be made while `stream` is being captured into a CUDA graph.
+ *   - Errors in arguments are reported before anything is launched.  No
+ *     entry point traps or aborts.
+ */
+#ifndef LF_ATTN_H
+#define LF_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { LF_F32 = 0, LF_BF16 = 1 } lf_dtype;
+
+typedef enum {
+    LF_OK = 0,
+    LF_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, bad dil/r/n_global */
+    LF_ERR_UNSUPPORTED = 2,  /* valid but outside what this build implements (see lf_attn_fwd) */
+    LF_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed */
+    LF_ERR_NO_MEMORY = 4,    /* workspace could not be allocated (or not during capture) */
+    LF_ERR_DEVICE_CHECK = 5  /* a device-side check fired (see lf_attn_device_status) */
+} lf_status;
+
+/*
+ * lf_attn_fwd -- the forward pass, asynchronous on `stream`.
+ *
+ *   q, k, v     device, [B,H,T,d], dtype `dtype`
+ *   out         device, [B,H,T,d], dtype `dtype`; fully overwritten
+ *   B, H, T, d  sizes (all >= 1)
+ *   r           one-sided window radius, w = 2r + 1, r >= 0
+ *   dil         HOST int32 [H], per-head dilation, each >= 1; NULL = all 1
+ *   global_idx  DEVICE int32 [B, n_global]: global positions per sample, any
+ *               order, duplicates allowed; NULL iff n_global == 0.  Entries
+ *               outside [0, T) are ignored and flagged in the device status.
+ *   n_global    >= 0
+ *   key_pad_mask DEVICE uint8 [B, T], nonzero = padded key; NULL = none
+ *   scale       softmax scale (usually 1/sqrt(d))
+ *   dtype       LF_F32: CUDA-core fp32 path, d <= 128.
+ *               LF_BF16: tensor-core path (tcgen05 + TMA), d == 64 only,
+ *               fp32 accumulation and softmax, every dil[h] <= 8, at most 4
+ *               distinct dilation values, H <= 128.
+ *   stream      a cudaStream_t (NULL = legacy default stream)
+ *
+ * Returns LF_OK once the kernels are queued; nothing is synchronised.
+ */
+lf_status lf_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                      int B, int H, int T, int d, int r, const int32_t* dil,
+                      const int32_t* global_idx, int n_global,
+                      const uint8_t* key_pad_mask, float scale, lf_dtype dtype,
+                      void* stream);
+
+/*
+ * lf_attn_fwd_host -- the same forward on HOST buffers.
+ *
+ * q, k, v, out, global_idx and key_pad_mask are host pointers with the
+ * layouts above (page-locked memory gives full copy bandwidth).  The call
+ * copies the inputs into a library-owned device staging area on `stream`,
+ * runs lf_attn_fwd, copies `out` back and synchronises `stream`, so `out`
+ * is ready when it returns.
+ */
+lf_status lf_attn_fwd_host(const void* q, const void* k, const void* v, void* out,
+                           int B, int H, int T, int d, int r, const int32_t* dil,
+                           const int32_t* global_idx, int n_global,
+                           const uint8_t* key_pad_mask, float scale, lf_dtype dtype,
+                           void* stream);
+
+/*
+ * lf_attn_fwd_stages -- runs a subset of the kernels lf_attn_fwd queues, for
+ * timing one kernel at a time.  Same arguments as lf_attn_fwd, plus
+ * stage_mask: bit 0 = prep (global lists, padding, packed global keys),
+ * bit 1 = band rows, bit 2 = global rows.  The band and global-row stages
+ * read what the prep stage of an earlier call with the same sizes,
+ * global_idx, key_pad_mask and k/v values left in the workspace; results
+ * are only defined when that holds.  stage_mask == 7 is lf_attn_fwd.
+ */
+lf_status lf_attn_fwd_stages(const void* q, const void* k, const void* v, void* out,
+                             int B, int H, int T, int d, int r, const int32_t* dil,
+                             const int32_t* global_idx, int n_global,
+                             const uint8_t* key_pad_mask, float scale, lf_dtype dtype,
+                             void* stream, uint32_t stage_mask);
+
+/*
+ * lf_attn_device_status -- synchronises `stream`, then reads and clears the
+ * current device's status word.  Returns LF_ERR_DEVICE_CHECK if a kernel
+ * since the last read flagged a data error (a global_idx entry outside
+ * [0, T)) or gave up waiting on one of its own pipeline barriers; `flags`
+ * (may be NULL) receives the raw bits:
+ *   bit 0  global_idx entry out of range (ignored by the computation)
+ *   bit 1  a pipeline wait timed out; that call's output is incomplete
+ */
+lf_status lf_attn_device_status(void* stream, uint32_t* flags);
+
+/* Text for a status code (static storage). */
+const char* lf_attn_strerror(lf_status status);
+
+/* Frees the workspaces of every device this process used. */
+void lf_attn_release(void);
+
+/* Bytes of device workspace lf_attn_fwd needs for these sizes. */
+uint64_t lf_attn_workspace_bytes(int B, int H, int T, int d, int n_global, lf_dtype dtype);
+
+/* Kernels launched by the last successful lf_attn_fwd on this host thread. */
+int lf_attn_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LF_ATTN_H */

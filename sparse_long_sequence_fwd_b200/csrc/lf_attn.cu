@@ -1,0 +1,474 @@
+// lf_attn.cu -- host side of liblfattn: argument checks, per-device
+// workspace, TMA tensor maps and the launch sequence
+//   K0 prep  ->  K1 band (bf16, tensor cores) | K3 band (fp32, CUDA cores)
+//            ->  K2 global rows (only when n_global > 0)
+// all on the caller's stream, nothing synchronised.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "lf_attn.h"
+#include "band_f32.cuh"
+#include "band_tc.cuh"
+#include "global_rows.cuh"
+#include "lf_common.cuh"
+#include "prep.cuh"
+
+namespace {
+
+using namespace lf;
+
+constexpr int kMaxDevices = 64;
+constexpr double kLog2e = 1.4426950408889634;
+
+struct DeviceState {
+    bool init = false;
+    int sm_count = 0;
+    uint32_t* status = nullptr;  // persistent device status word
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+    void* io = nullptr;  // staging for lf_attn_fwd_host
+    size_t io_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+thread_local int t_last_launches = 0;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Layout {
+    size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, total;
+    int W, gstride, nchunk, ngp;
+};
+
+Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
+    Layout L{};
+    L.W = (T + 31) / 32;
+    L.gstride = std::max(1, std::min(n_global, T));
+    L.nchunk = (T + kChunk - 1) / kChunk;
+    L.ngp = (L.gstride + 15) & ~15;
+    size_t o = 0;
+    L.off_ngq = o; o = align256(o + sizeof(int32_t) * B);
+    L.off_ngk = o; o = align256(o + sizeof(int32_t) * B);
+    L.off_gq = o; o = align256(o + sizeof(int32_t) * size_t(B) * L.gstride);
+    L.off_gk = o; o = align256(o + sizeof(int32_t) * size_t(B) * L.gstride);
+    L.off_gbit = o; o = align256(o + sizeof(uint32_t) * size_t(B) * L.W);
+    L.off_cnt = o; o = align256(o + sizeof(int32_t) * size_t(B) * H);
+    L.off_part = o;
+    if (n_global > 0) o = align256(o + sizeof(float) * size_t(B) * H * L.gstride * L.nchunk * (d + 2));
+    L.off_kg = o;
+    L.off_vg = o;
+    if (dtype == LF_BF16 && n_global > 0) {
+        const size_t kgb = sizeof(__nv_bfloat16) * size_t(B) * H * L.ngp * 64;
+        L.off_vg = align256(o + kgb);
+        o = align256(L.off_vg + kgb);
+    }
+    L.total = std::max<size_t>(o, 256);
+    return L;
+}
+
+bool is_capturing(cudaStream_t s) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &st) != cudaSuccess) return false;
+    return st != cudaStreamCaptureStatusNone;
+}
+
+lf_status device_state(DeviceState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_CUDA;
+    DeviceState& s = g_dev[dev];
+    if (!s.init) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LF_ERR_CUDA;
+        if (prop.major < 10) return LF_ERR_UNSUPPORTED;
+        s.sm_count = prop.multiProcessorCount;
+        if (cudaMalloc(&s.status, 256) != cudaSuccess) return LF_ERR_NO_MEMORY;
+        if (cudaMemset(s.status, 0, 256) != cudaSuccess) return LF_ERR_CUDA;
+        if (cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) !=
+            cudaSuccess)
+            return LF_ERR_CUDA;
+        const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + kMaxGlobal) * 4;
+        if (cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) !=
+            cudaSuccess)
+            return LF_ERR_CUDA;
+        const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
+        if (cudaFuncSetAttribute(global_rows_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gr_max) != cudaSuccess ||
+            cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gr_max) != cudaSuccess ||
+            cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gr_max) != cudaSuccess ||
+            cudaFuncSetAttribute(global_rows_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGrBf16Smem) != cudaSuccess)
+            return LF_ERR_CUDA;
+        s.init = true;
+    }
+    *out = &s;
+    return LF_OK;
+}
+
+lf_status grow(void** buf, size_t* have, size_t need, cudaStream_t stream) {
+    if (*have >= need) return LF_OK;
+    if (is_capturing(stream)) return LF_ERR_NO_MEMORY;
+    if (*buf) {
+        cudaFree(*buf);  // synchronises the device: no kernel still uses it
+        *buf = nullptr;
+        *have = 0;
+    }
+    if (cudaMalloc(buf, need) != cudaSuccess) {
+        *buf = nullptr;
+        return LF_ERR_NO_MEMORY;
+    }
+    if (cudaMemset(*buf, 0, need) != cudaSuccess) return LF_ERR_CUDA;
+    *have = need;
+    return LF_OK;
+}
+
+lf_status get_encoder() {
+    if (g_encode) return LF_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return LF_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return LF_OK;
+}
+
+// 3-D bf16 map over [d=64, rows, B*H] with a 128-byte swizzle; box = 64 x
+// (rows_per_box * stride) x 1, element stride `stride` along the rows.
+lf_status encode_rows_map(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t bh, uint32_t rows_per_box,
+                          uint32_t stride) {
+    cuuint64_t gdim[3] = {64, rows, bh};
+    cuuint64_t gstr[2] = {64 * 2, rows * 64 * 2};
+    cuuint32_t box[3] = {64, rows_per_box * stride, 1};
+    cuuint32_t estr[3] = {1, stride, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstr, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LF_OK : LF_ERR_CUDA;
+}
+
+lf_status check_args(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d, int r,
+                     const int32_t* dil, const int32_t* gidx, int n_global, float scale, lf_dtype dtype) {
+    if (!q || !k || !v || !out) return LF_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || r < 0 || n_global < 0) return LF_ERR_INVALID_ARG;
+    if (n_global > 0 && !gidx) return LF_ERR_INVALID_ARG;
+    if (n_global == 0 && gidx) return LF_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return LF_ERR_INVALID_ARG;
+    if (dtype != LF_F32 && dtype != LF_BF16) return LF_ERR_INVALID_ARG;
+    if (dil)
+        for (int h = 0; h < H; ++h)
+            if (dil[h] < 1) return LF_ERR_INVALID_ARG;
+    const uint64_t n = uint64_t(B) * uint64_t(H) * uint64_t(T) * uint64_t(d);
+    if (n / uint64_t(d) / uint64_t(T) / uint64_t(H) != uint64_t(B) || n > (uint64_t(1) << 40))
+        return LF_ERR_INVALID_ARG;
+    for (const void* p : {q, k, v, static_cast<const void*>(out)})
+        if (reinterpret_cast<uintptr_t>(p) & 15u) return LF_ERR_INVALID_ARG;
+    if (T > kMaxT || n_global > kMaxGlobal) return LF_ERR_UNSUPPORTED;
+    if (uint64_t(B) * H > 0x7fffffffull || uint64_t(B) * H * T > (uint64_t(1) << 31) * 64) return LF_ERR_UNSUPPORTED;
+    if (dtype == LF_F32 && d > 128) return LF_ERR_UNSUPPORTED;
+    if (n_global > 0 && uint64_t(B) * H > 65535u) return LF_ERR_UNSUPPORTED;  // global-row grid.y
+    if (dtype == LF_BF16) {
+        if (d != 64 || H > kMaxHeads) return LF_ERR_UNSUPPORTED;
+        int kinds[kMaxDilKinds];
+        int nk = 0;
+        for (int h = 0; h < H; ++h) {
+            const int dl = dil ? dil[h] : 1;
+            if (dl > kMaxDilTma) return LF_ERR_UNSUPPORTED;
+            bool seen = false;
+            for (int a = 0; a < nk; ++a) seen |= kinds[a] == dl;
+            if (!seen) {
+                if (nk == kMaxDilKinds) return LF_ERR_UNSUPPORTED;
+                kinds[nk++] = dl;
+            }
+        }
+    }
+    return LF_OK;
+}
+
+lf_status launch_all(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d, int r,
+                     const int32_t* dil, const int32_t* gidx, int n_global, const uint8_t* pad, float scale,
+                     lf_dtype dtype, cudaStream_t stream, DeviceState* ds, uint32_t stages = 7u) {
+    const Layout L = make_layout(B, H, T, d, n_global, dtype);
+    lf_status st = grow(&ds->ws, &ds->ws_bytes, L.total, stream);
+    if (st != LF_OK) return st;
+    uint8_t* base = static_cast<uint8_t*>(ds->ws);
+    Workspace ws;
+    ws.n_gq = reinterpret_cast<int32_t*>(base + L.off_ngq);
+    ws.n_gk = reinterpret_cast<int32_t*>(base + L.off_ngk);
+    ws.gq_list = reinterpret_cast<int32_t*>(base + L.off_gq);
+    ws.gk_list = reinterpret_cast<int32_t*>(base + L.off_gk);
+    ws.gbit = reinterpret_cast<uint32_t*>(base + L.off_gbit);
+    ws.counters = reinterpret_cast<int32_t*>(base + L.off_cnt);
+    ws.partial = reinterpret_cast<float*>(base + L.off_part);
+    ws.kg = reinterpret_cast<__nv_bfloat16*>(base + L.off_kg);
+    ws.vg = reinterpret_cast<__nv_bfloat16*>(base + L.off_vg);
+    const int r_eff = std::min(r, T);  // a window wider than the sequence changes nothing
+    const float sl2 = static_cast<float>(double(scale) * kLog2e);
+    int launches = 0;
+
+    // K0
+    PrepParams pp;
+    pp.gidx = gidx;
+    pp.pad = pad;
+    pp.k = k;
+    pp.v = v;
+    pp.ws = ws;
+    pp.status = ds->status;
+    pp.B = B; pp.H = H; pp.T = T; pp.d = d;
+    pp.n_global = n_global;
+    pp.gstride = L.gstride;
+    pp.ngp = L.ngp;
+    pp.W = L.W;
+    pp.pack = (dtype == LF_BF16 && n_global > 0) ? 1 : 0;
+    const size_t prep_smem = size_t(L.W + 2 * kPrepThreads + L.gstride) * 4;
+    if (stages & 1u) {
+        prep_kernel<<<B * H, kPrepThreads, prep_smem, stream>>>(pp);
+        ++launches;
+    }
+
+    if (!(stages & 2u)) {
+        // band stage skipped
+    } else if (dtype == LF_F32) {
+        // K3: fp32 band rows on CUDA cores
+        BandF32Params bp;
+        bp.q = static_cast<const float*>(q);
+        bp.k = static_cast<const float*>(k);
+        bp.v = static_cast<const float*>(v);
+        bp.out = static_cast<float*>(out);
+        bp.pad = pad;
+        bp.ws = ws;
+        bp.B = B; bp.H = H; bp.T = T; bp.d = d; bp.r = r_eff;
+        bp.gstride = L.gstride;
+        bp.W = L.W;
+        bp.sl2 = sl2;
+        for (int h = 0; h < kMaxHeads; ++h) bp.dil[h] = (h < H && dil) ? dil[h] : 1;
+        const long rows = long(B) * H * T;
+        const unsigned grid = static_cast<unsigned>((rows + kBandF32Warps - 1) / kBandF32Warps);
+        if (d <= 16) band_f32_kernel<16><<<grid, kBandF32Warps * 32, 0, stream>>>(bp);
+        else if (d <= 32) band_f32_kernel<32><<<grid, kBandF32Warps * 32, 0, stream>>>(bp);
+        else if (d <= 64) band_f32_kernel<64><<<grid, kBandF32Warps * 32, 0, stream>>>(bp);
+        else band_f32_kernel<128><<<grid, kBandF32Warps * 32, 0, stream>>>(bp);
+        ++launches;
+    } else {
+        // K1: bf16 band rows on the tensor cores
+        st = get_encoder();
+        if (st != LF_OK) return st;
+        static thread_local BandTcParams bp;  // large (tensor maps); filled per call
+        std::memset(&bp, 0, sizeof(bp));
+        int nk = 0;
+        int kind_of_head[kMaxHeads];
+        for (int h = 0; h < H; ++h) {
+            const int dl = dil ? dil[h] : 1;
+            int kidx = -1;
+            for (int a = 0; a < nk; ++a)
+                if (bp.dk_dil[a] == dl) kidx = a;
+            if (kidx < 0) {
+                kidx = nk++;
+                bp.dk_dil[kidx] = dl;
+                bp.dk_rows[kidx] = dl <= 2 ? 128 : (dl <= 4 ? 64 : 32);
+                const uint32_t R = static_cast<uint32_t>(bp.dk_rows[kidx]);
+                if ((st = encode_rows_map(&bp.tm_q[kidx], q, T, uint64_t(B) * H, R, dl)) != LF_OK ||
+                    (st = encode_rows_map(&bp.tm_k[kidx], k, T, uint64_t(B) * H, R, dl)) != LF_OK ||
+                    (st = encode_rows_map(&bp.tm_v[kidx], v, T, uint64_t(B) * H, R, dl)) != LF_OK)
+                    return st;
+            }
+            kind_of_head[h] = kidx;
+        }
+        for (int a = nk; a < kMaxDilKinds; ++a) {  // unused slots: valid maps, never read
+            bp.tm_q[a] = bp.tm_q[0];
+            bp.tm_k[a] = bp.tm_k[0];
+            bp.tm_v[a] = bp.tm_v[0];
+            bp.dk_dil[a] = 1;
+            bp.dk_rows[a] = 128;
+        }
+        if (n_global > 0) {
+            if ((st = encode_rows_map(&bp.tm_kg, ws.kg, L.ngp, uint64_t(B) * H, 128, 1)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_vg, ws.vg, L.ngp, uint64_t(B) * H, 128, 1)) != LF_OK)
+                return st;
+        } else {
+            bp.tm_kg = bp.tm_k[0];
+            bp.tm_vg = bp.tm_v[0];
+        }
+        int items_per_b = 0;
+        for (int h = 0; h < H; ++h) {
+            bp.head_start[h] = items_per_b;
+            bp.head_dk[h] = static_cast<uint8_t>(kind_of_head[h]);
+            const int dl = bp.dk_dil[kind_of_head[h]];
+            for (int c = 0; c < dl; ++c) {
+                const int Tc = (T - c + dl - 1) / dl;
+                items_per_b += (Tc + kBM - 1) / kBM;
+            }
+        }
+        for (int h = H; h <= kMaxHeads; ++h) bp.head_start[h] = items_per_b;
+        bp.out = static_cast<__nv_bfloat16*>(out);
+        bp.pad = pad;
+        bp.gk_list = ws.gk_list;
+        bp.n_gk = ws.n_gk;
+        bp.gbit = ws.gbit;
+        bp.status = ds->status;
+        bp.B = B; bp.H = H; bp.T = T; bp.r = r_eff;
+        bp.W = L.W;
+        bp.gstride = L.gstride;
+        bp.sl2 = sl2;
+        bp.items_per_b = items_per_b;
+        bp.n_items = items_per_b * B;
+        const int grid = std::min(bp.n_items, ds->sm_count);
+        band_tc_kernel<<<grid, kBandThreads, kBandSmem, stream>>>(bp);
+        ++launches;
+    }
+
+    if (n_global > 0 && (stages & 4u)) {
+        // K2: rows of the global queries
+        GlobalRowParams gp;
+        gp.q = q;
+        gp.k = k;
+        gp.v = v;
+        gp.out = out;
+        gp.pad = pad;
+        gp.ws = ws;
+        gp.B = B; gp.H = H; gp.T = T; gp.d = d;
+        gp.gstride = L.gstride;
+        gp.nchunk = L.nchunk;
+        gp.sl2 = sl2;
+        const dim3 grid(L.nchunk, B * H);
+        const int DP = d <= 32 ? 32 : (d <= 64 ? 64 : 128);
+        const size_t smem = size_t(kChunk * DP + DP + kChunk + 32 + kGrThreads) * 4;
+        if (dtype == LF_BF16) global_rows_bf16_kernel<<<grid, kGrThreads, kGrBf16Smem, stream>>>(gp);
+        else if (DP == 32) global_rows_kernel<float, 32><<<grid, kGrThreads, smem, stream>>>(gp);
+        else if (DP == 64) global_rows_kernel<float, 64><<<grid, kGrThreads, smem, stream>>>(gp);
+        else global_rows_kernel<float, 128><<<grid, kGrThreads, smem, stream>>>(gp);
+        ++launches;
+    }
+    if (cudaGetLastError() != cudaSuccess) return LF_ERR_CUDA;
+    t_last_launches = launches;
+    return LF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lf_status lf_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d, int r,
+                      const int32_t* dil, const int32_t* global_idx, int n_global, const uint8_t* key_pad_mask,
+                      float scale, lf_dtype dtype, void* stream) {
+    lf_status st = check_args(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, scale, dtype);
+    if (st != LF_OK) return st;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    if ((st = device_state(&ds)) != LF_OK) return st;
+    return launch_all(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, key_pad_mask, scale, dtype,
+                      static_cast<cudaStream_t>(stream), ds);
+}
+
+lf_status lf_attn_fwd_stages(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d,
+                             int r, const int32_t* dil, const int32_t* global_idx, int n_global,
+                             const uint8_t* key_pad_mask, float scale, lf_dtype dtype, void* stream,
+                             uint32_t stage_mask) {
+    lf_status st = check_args(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, scale, dtype);
+    if (st != LF_OK) return st;
+    if (stage_mask == 0u || stage_mask > 7u) return LF_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    if ((st = device_state(&ds)) != LF_OK) return st;
+    return launch_all(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, key_pad_mask, scale, dtype,
+                      static_cast<cudaStream_t>(stream), ds, stage_mask);
+}
+
+lf_status lf_attn_fwd_host(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d,
+                           int r, const int32_t* dil, const int32_t* global_idx, int n_global,
+                           const uint8_t* key_pad_mask, float scale, lf_dtype dtype, void* stream) {
+    lf_status st = check_args(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, scale, dtype);
+    if (st != LF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    if ((st = device_state(&ds)) != LF_OK) return st;
+    const size_t es = dtype == LF_BF16 ? 2 : 4;
+    const size_t nb = size_t(B) * H * T * d * es;
+    const size_t o_q = 0, o_k = align256(nb), o_v = 2 * align256(nb), o_o = 3 * align256(nb);
+    const size_t o_g = 4 * align256(nb);
+    const size_t o_p = o_g + align256(sizeof(int32_t) * size_t(B) * std::max(n_global, 1));
+    const size_t total = o_p + align256(size_t(B) * T);
+    if ((st = grow(&ds->io, &ds->io_bytes, total, s)) != LF_OK) return st;
+    uint8_t* io = static_cast<uint8_t*>(ds->io);
+    if (cudaMemcpyAsync(io + o_q, q, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(io + o_k, k, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(io + o_v, v, nb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return LF_ERR_CUDA;
+    if (n_global > 0 &&
+        cudaMemcpyAsync(io + o_g, global_idx, sizeof(int32_t) * size_t(B) * n_global, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess)
+        return LF_ERR_CUDA;
+    if (key_pad_mask && cudaMemcpyAsync(io + o_p, key_pad_mask, size_t(B) * T, cudaMemcpyHostToDevice, s) !=
+                            cudaSuccess)
+        return LF_ERR_CUDA;
+    st = launch_all(io + o_q, io + o_k, io + o_v, io + o_o, B, H, T, d, r, dil,
+                    n_global > 0 ? reinterpret_cast<const int32_t*>(io + o_g) : nullptr, n_global,
+                    key_pad_mask ? io + o_p : nullptr, scale, dtype, s, ds);
+    if (st != LF_OK) return st;
+    if (cudaMemcpyAsync(out, io + o_o, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return LF_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LF_ERR_CUDA;
+    return LF_OK;
+}
+
+lf_status lf_attn_device_status(void* stream, uint32_t* flags) {
+    if (flags) *flags = 0;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LF_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    lf_status st = device_state(&ds);
+    if (st != LF_OK) return st;
+    uint32_t h = 0;
+    if (cudaMemcpy(&h, ds->status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return LF_ERR_CUDA;
+    if (cudaMemset(ds->status, 0, sizeof(h)) != cudaSuccess) return LF_ERR_CUDA;
+    if (flags) *flags = h;
+    return h ? LF_ERR_DEVICE_CHECK : LF_OK;
+}
+
+const char* lf_attn_strerror(lf_status s) {
+    switch (s) {
+        case LF_OK: return "ok";
+        case LF_ERR_INVALID_ARG: return "invalid argument";
+        case LF_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case LF_ERR_CUDA: return "CUDA error";
+        case LF_ERR_NO_MEMORY: return "workspace allocation failed (or attempted during stream capture)";
+        case LF_ERR_DEVICE_CHECK: return "device-side check failed";
+    }
+    return "unknown status";
+}
+
+void lf_attn_release(void) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (int dev = 0; dev < kMaxDevices; ++dev) {
+        DeviceState& s = g_dev[dev];
+        if (!s.init) continue;
+        cudaSetDevice(dev);
+        if (s.ws) cudaFree(s.ws);
+        if (s.io) cudaFree(s.io);
+        if (s.status) cudaFree(s.status);
+        s = DeviceState();
+    }
+    cudaSetDevice(cur);
+}
+
+uint64_t lf_attn_workspace_bytes(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
+    if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || n_global < 0) return 0;
+    return make_layout(B, H, T, d, n_global, dtype).total;
+}
+
+int lf_attn_last_launch_count(void) { return t_last_launches; }
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// lf_common.cuh -- limits, device status bits and kernel parameter blocks
+// shared by the host launcher and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+namespace lf {
+
+constexpr int kMaxHeads = 128;      // H limit (per-head tables travel in the kernel parameters)
+constexpr int kMaxDilKinds = 4;     // distinct dilation values per call (tensor-core path)
+constexpr int kMaxDilTma = 8;       // TMA element stride limit
+constexpr int kMaxT = 1 << 20;      // sequence length limit (prep bitmap lives in shared memory)
+constexpr int kMaxGlobal = 4096;    // n_global limit
+constexpr int kChunk = 256;         // keys per CTA in the global-row kernel
+
+// device status word bits
+constexpr uint32_t kStatusBadGlobal = 1u;  // a global_idx entry outside [0, T)
+constexpr uint32_t kStatusTimeout = 2u;    // a pipeline wait gave up
+
+// Workspace carved by the host (all offsets 256-byte aligned).
+struct Workspace {
+    int32_t* n_gq;      // [B]      in-range unique global queries
+    int32_t* n_gk;      // [B]      ... of which not padded (global keys)
+    int32_t* gq_list;   // [B][gstride] sorted
+    int32_t* gk_list;   // [B][gstride] sorted
+    uint32_t* gbit;     // [B][W]   bit i = position i is a global query
+    int32_t* counters;  // [B*H]    arrival tickets of the global-row kernel (kept at 0 between calls)
+    float* partial;     // [B*H][gstride][nchunk][d + 2]
+    __nv_bfloat16* kg;  // [B*H][ngp][64] packed global keys (bf16 path)
+    __nv_bfloat16* vg;  // [B*H][ngp][64] packed global values
+};
+
+struct PrepParams {
+    const int32_t* gidx;  // [B][n_global] or null
+    const uint8_t* pad;   // [B][T] or null
+    const void* k;        // [B,H,T,d] (bf16 path: packed into kg)
+    const void* v;
+    Workspace ws;
+    uint32_t* status;
+    int B, H, T, d, n_global, gstride, ngp, W;
+    int pack;             // 1: write kg/vg (bf16, d == 64)
+};
+
+struct GlobalRowParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* out;
+    const uint8_t* pad;
+    Workspace ws;
+    int B, H, T, d, gstride, nchunk;
+    float sl2;  // scale * log2(e)
+};
+
+struct BandF32Params {
+    const float* q;
+    const float* k;
+    const float* v;
+    float* out;
+    const uint8_t* pad;
+    Workspace ws;
+    int B, H, T, d, r, gstride, W;
+    float sl2;
+    int dil[kMaxHeads];  // per-head dilation
+};
+
+struct BandTcParams {
+    CUtensorMap tm_q[kMaxDilKinds];
+    CUtensorMap tm_k[kMaxDilKinds];
+    CUtensorMap tm_v[kMaxDilKinds];
+    CUtensorMap tm_kg;
+    CUtensorMap tm_vg;
+    __nv_bfloat16* out;
+    const uint8_t* pad;
+    const int32_t* gk_list;
+    const int32_t* n_gk;
+    const uint32_t* gbit;
+    uint32_t* status;
+    int B, H, T, r, W, gstride;
+    float sl2;
+    int n_items;     // work items (b, h, residue class, 128-query tile)
+    int items_per_b;
+    int dk_dil[kMaxDilKinds];
+    int dk_rows[kMaxDilKinds];   // rows per TMA box for that dilation
+    int head_start[kMaxHeads + 1];  // item offset of each head inside one sample
+    uint8_t head_dk[kMaxHeads];
+};
+
+}  // namespace lf

@@ -1,0 +1,128 @@
+// prep.cuh -- K0: global-token and padding preparation.
+//
+// One CTA per (b, h).  From global_idx[b, :] it builds the set G_b (in-range
+// entries, duplicates collapsed) as a bitmap in shared memory, then the
+// sorted lists
+//   gq_list[b] = G_b                       (global queries: full rows)
+//   gk_list[b] = G_b minus padded keys     (global keys: extra columns)
+// and the global-query bitmap gbit[b].  Set semantics follow the "Longformer"
+// note, section "Global Attention" (N(i) = N_local(i) U G); a padded position
+// is removed as a key ("Implementation Reading": padding must be masked) but
+// is still a global query.  Entries outside [0, T) are ignored and raise the
+// status bit.  It also zeroes the arrival counters the global-row kernel
+// uses for its (b, h).  On the bf16 path every CTA also packs the rows of k and v
+// named by gk_list into contiguous [ngp][64] blocks for its (b, h), zero
+// beyond the list, so the band kernel can stage them with one TMA box.
+#pragma once
+#include "lf_common.cuh"
+
+namespace lf {
+
+constexpr int kPrepThreads = 256;
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* sbuf) {
+    // sbuf: kPrepThreads ints; returns exclusive prefix, leaves the total in sbuf[kPrepThreads-1] + v_last
+    const int tid = threadIdx.x;
+    sbuf[tid] = v;
+    __syncthreads();
+    for (int off = 1; off < kPrepThreads; off <<= 1) {
+        int t = tid >= off ? sbuf[tid - off] : 0;
+        __syncthreads();
+        sbuf[tid] += t;
+        __syncthreads();
+    }
+    int incl = sbuf[tid];
+    return incl - v;
+}
+
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
+    extern __shared__ __align__(16) uint32_t prep_smem[];
+    uint32_t* bits = prep_smem;                                      // [W]
+    int* scan_q = reinterpret_cast<int*>(bits + p.W);                // [256]
+    int* scan_k = scan_q + kPrepThreads;                             // [256]
+    int* gk_s = scan_k + kPrepThreads;                               // [gstride]
+    __shared__ int n_k_total;
+
+    const int tid = threadIdx.x;
+    const int b = blockIdx.x / p.H;
+    const int h = blockIdx.x - b * p.H;
+    const int T = p.T;
+    const uint8_t* pad_b = p.pad ? p.pad + static_cast<size_t>(b) * T : nullptr;
+
+    for (int w = tid; w < p.W; w += kPrepThreads) bits[w] = 0u;
+    if (tid == 0) p.ws.counters[blockIdx.x] = 0;  // arrival tickets of the global-row kernel
+    __syncthreads();
+    for (int a = tid; a < p.n_global; a += kPrepThreads) {
+        int g = p.gidx[static_cast<size_t>(b) * p.n_global + a];
+        if (g < 0 || g >= T) {
+            if (h == 0) atomicOr(p.status, kStatusBadGlobal);
+        } else {
+            atomicOr(&bits[g >> 5], 1u << (g & 31));
+        }
+    }
+    __syncthreads();
+
+    // contiguous word range per thread
+    const int per = (p.W + kPrepThreads - 1) / kPrepThreads;
+    const int w0 = min(p.W, tid * per), w1 = min(p.W, w0 + per);
+    int cq = 0, ck = 0;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t qb = bits[w];
+        cq += __popc(qb);
+        uint32_t kb = qb;
+        if (pad_b) {
+            for (uint32_t t = qb; t; t &= t - 1) {
+                int j = (w << 5) + __ffs(t) - 1;
+                if (pad_b[j]) kb &= ~(1u << (j & 31));
+            }
+        }
+        ck += __popc(kb);
+    }
+    int oq = block_exclusive_scan(cq, scan_q);
+    int ok = block_exclusive_scan(ck, scan_k);
+    if (tid == kPrepThreads - 1) n_k_total = ok + ck;
+    const bool writer = (h == 0);
+    int32_t* gq_out = p.ws.gq_list + static_cast<size_t>(b) * p.gstride;
+    int32_t* gk_out = p.ws.gk_list + static_cast<size_t>(b) * p.gstride;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t qb = bits[w];
+        if (writer) p.ws.gbit[static_cast<size_t>(b) * p.W + w] = qb;
+        for (uint32_t t = qb; t; t &= t - 1) {
+            int j = (w << 5) + __ffs(t) - 1;
+            if (writer) gq_out[oq] = j;
+            ++oq;
+            if (!pad_b || !pad_b[j]) {
+                gk_s[ok] = j;
+                if (writer) gk_out[ok] = j;
+                ++ok;
+            }
+        }
+    }
+    if (writer && tid == kPrepThreads - 1) {
+        p.ws.n_gq[b] = oq;
+        p.ws.n_gk[b] = ok;
+    }
+    __syncthreads();
+
+    if (p.pack) {
+        const int nk = n_k_total;
+        const size_t bh = static_cast<size_t>(b) * p.H + h;
+        const uint4* k4 = reinterpret_cast<const uint4*>(p.k) + bh * T * 8;
+        const uint4* v4 = reinterpret_cast<const uint4*>(p.v) + bh * T * 8;
+        uint4* kg4 = reinterpret_cast<uint4*>(p.ws.kg) + bh * p.ngp * 8;
+        uint4* vg4 = reinterpret_cast<uint4*>(p.ws.vg) + bh * p.ngp * 8;
+        for (int idx = tid; idx < p.ngp * 8; idx += kPrepThreads) {
+            int a = idx >> 3, c = idx & 7;
+            uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+            if (a < nk) {
+                size_t row = static_cast<size_t>(gk_s[a]);
+                kv = k4[row * 8 + c];
+                vv = v4[row * 8 + c];
+            }
+            kg4[idx] = kv;
+            vg4[idx] = vv;
+        }
+    }
+}
+
+}  // namespace lf

@@ -1,0 +1,182 @@
+"""ctypes binding of liblfattn (``include/lf_attn.h``): argument marshalling only.
+
+Every step of the forward runs in the library's CUDA kernels.  There is no
+fallback: if the shared library is missing or cannot be loaded, the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblfattn.so")
+
+LF_F32, LF_BF16 = 0, 1
+STATUS = {0: "LF_OK", 1: "LF_ERR_INVALID_ARG", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
+          4: "LF_ERR_NO_MEMORY", 5: "LF_ERR_DEVICE_CHECK"}
+EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
+           "lf_attn_release", "lf_attn_workspace_bytes", "lf_attn_last_launch_count")
+
+_lib = None
+
+
+class LfAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s (%s)" % (what, STATUS.get(status, status), strerror(status)))
+
+
+def load():
+    """Load liblfattn.so (built in-tree by build.py); raises if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("liblfattn.so is not built (run sparse_long_sequence_fwd_b200/build.py)")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        sig = [P, P, P, P, I, I, I, I, I, P, P, I, P, ctypes.c_float, I, P]
+        lib.lf_attn_fwd.argtypes = sig
+        lib.lf_attn_fwd.restype = I
+        lib.lf_attn_fwd_stages.argtypes = sig + [ctypes.c_uint32]
+        lib.lf_attn_fwd_stages.restype = I
+        lib.lf_attn_fwd_host.argtypes = sig
+        lib.lf_attn_fwd_host.restype = I
+        lib.lf_attn_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+        lib.lf_attn_device_status.restype = I
+        lib.lf_attn_strerror.argtypes = [I]
+        lib.lf_attn_strerror.restype = ctypes.c_char_p
+        lib.lf_attn_release.argtypes = []
+        lib.lf_attn_release.restype = None
+        lib.lf_attn_workspace_bytes.argtypes = [I, I, I, I, I, I]
+        lib.lf_attn_workspace_bytes.restype = ctypes.c_uint64
+        lib.lf_attn_last_launch_count.argtypes = []
+        lib.lf_attn_last_launch_count.restype = I
+        _lib = lib
+    return _lib
+
+
+def strerror(status: int) -> str:
+    try:
+        return load().lf_attn_strerror(int(status)).decode()
+    except Exception:  # library absent: still format the error
+        return STATUS.get(status, "unknown")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LF_F32
+    if t.dtype == torch.bfloat16:
+        return LF_BF16
+    raise TypeError("q/k/v must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _dil_array(dil, H):
+    if dil is None:
+        return None
+    if isinstance(dil, int):
+        dil = [dil] * H
+    vals = [int(x) for x in (dil.tolist() if hasattr(dil, "tolist") else dil)]
+    if len(vals) != H:
+        raise ValueError("dil must have H entries")
+    return (ctypes.c_int32 * H)(*vals)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_qkv(q, k, v):
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must all be [B, H, T, d]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, r: int, dil=None,
+        global_idx: Optional[torch.Tensor] = None, key_pad_mask: Optional[torch.Tensor] = None,
+        scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+        stream: Optional[torch.cuda.Stream] = None, stages: int = 7) -> torch.Tensor:
+    """lf_attn_fwd on CUDA tensors, queued on ``stream`` (default: current stream).
+
+    ``stages`` != 7 calls lf_attn_fwd_stages (per-kernel timing)."""
+    _check_qkv(q, k, v)
+    B, H, T, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    n_global = 0
+    if global_idx is not None:
+        if global_idx.dtype != torch.int32 or not global_idx.is_contiguous() or global_idx.dim() != 2:
+            raise ValueError("global_idx must be a contiguous int32 [B, n_global] tensor")
+        n_global = global_idx.shape[1]
+        if n_global == 0:
+            global_idx = None
+    if key_pad_mask is not None and (key_pad_mask.dtype != torch.uint8 or not key_pad_mask.is_contiguous()):
+        raise ValueError("key_pad_mask must be a contiguous uint8 [B, T] tensor")
+    if scale is None:
+        scale = d ** -0.5
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, d, int(r), _dil_array(dil, H),
+            _ptr(global_idx), n_global, _ptr(key_pad_mask), float(scale), _dtype_code(q),
+            ctypes.c_void_p(s.cuda_stream))
+    if stages == 7:
+        st = load().lf_attn_fwd(*args)
+    else:
+        st = load().lf_attn_fwd_stages(*args, ctypes.c_uint32(stages))
+    if st != 0:
+        raise LfAttnError(st, "lf_attn_fwd")
+    return out
+
+
+def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, r: int, dil=None,
+             global_idx: Optional[torch.Tensor] = None, key_pad_mask: Optional[torch.Tensor] = None,
+             scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """lf_attn_fwd_host on CPU tensors (pinned for full copy bandwidth); returns when ``out`` is ready."""
+    _check_qkv(q, k, v)
+    B, H, T, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    n_global = 0 if global_idx is None else global_idx.shape[1]
+    if n_global == 0:
+        global_idx = None
+    if scale is None:
+        scale = d ** -0.5
+    s = stream if stream is not None else torch.cuda.current_stream()
+    st = load().lf_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, d, int(r), _dil_array(dil, H),
+                                 _ptr(global_idx), n_global, _ptr(key_pad_mask), float(scale), _dtype_code(q),
+                                 ctypes.c_void_p(s.cuda_stream))
+    if st != 0:
+        raise LfAttnError(st, "lf_attn_fwd_host")
+    return out
+
+
+def device_status(stream: Optional[torch.cuda.Stream] = None):
+    """(status, flags): synchronises the stream, reads and clears the device status word."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    flags = ctypes.c_uint32(0)
+    st = load().lf_attn_device_status(ctypes.c_void_p(s.cuda_stream), ctypes.byref(flags))
+    return st, flags.value
+
+
+def release() -> None:
+    load().lf_attn_release()
+
+
+def workspace_bytes(B, H, T, d, n_global, dtype_code) -> int:
+    return int(load().lf_attn_workspace_bytes(B, H, T, d, n_global, dtype_code))
+
+
+def last_launch_count() -> int:
+    return int(load().lf_attn_last_launch_count())
+
+
+def raw_call(name: str, *args) -> int:
+    """Calls an entry point with raw arguments (used by the error-path tests)."""
+    return getattr(load(), name)(*args)

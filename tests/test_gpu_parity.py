@@ -1,0 +1,166 @@
+"""CUDA path vs the fp64 oracle, on the same seeded inputs.
+
+* tiny fp32 workload, every element, max-abs <= 1e-5;
+* small bf16 and fp32 cases that the oracle finishes in seconds but that
+  span several 128-row tiles, a ragged tail, several residue classes,
+  padding and more than one 128-wide block of global keys: every element;
+* the four full-size bf16 workloads in the launch configuration the bench
+  times: the base workload in full, the others on sampled rows;
+* edge cases: T < w, r = 0, no globals, global at T-1, padded globals,
+  an all-padded sample, T mod dil != 0, duplicates, out-of-range entries.
+bf16 bar: max-abs <= 2e-2 and relative RMS <= 5e-3 over the compared rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+from sparse_long_sequence_fwd_b200 import build, lf_attn, workloads
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    build.build()
+    lf_attn.load()
+    yield
+
+
+def _full_case(w):
+    inp = workloads.make_inputs(w)
+    got = parity.run_gpu(w, inp)
+    ref = parity.oracle_full(w, inp)
+    return parity.compare(w, got, ref)
+
+
+def test_tiny_f32_workload_every_element():
+    _full_case(workloads.TINY)
+
+
+SMALL = [
+    workloads.custom("bf16_multi_tile", "bf16", 2, 3, 1000, 64, 100, dil=[1, 2, 3],
+                     globals_per_b=[[0, 999, 500, 500], [7, 3, 3, 640]], pad_from=[None, 777], seed=11),
+    workloads.custom("bf16_r256_T1500", "bf16", 1, 2, 1500, 64, 256, dil=[1, 2],
+                     globals_per_b=[[0]], seed=12),
+    workloads.custom("bf16_many_globals", "bf16", 1, 2, 1200, 64, 64, dil=[1, 4],
+                     globals_per_b=[list(range(0, 1200, 4))], pad_from=[1100], seed=13),
+    workloads.custom("bf16_dil_5_to_8", "bf16", 1, 4, 700, 64, 20, dil=[5, 6, 7, 8],
+                     globals_per_b=[[1, 2, 699]], seed=14),
+    workloads.custom("f32_multi_tile", "f32", 2, 3, 600, 64, 70, dil=[1, 2, 3],
+                     globals_per_b=[[0, 599], [11, 11]], pad_from=[None, 450], seed=15),
+    workloads.custom("f32_d128", "f32", 1, 2, 300, 128, 40, dil=[1, 2], globals_per_b=[[5]], seed=16),
+    workloads.custom("f32_d24", "f32", 1, 2, 200, 24, 9, dil=[3, 1], globals_per_b=[[0, 100]], seed=17),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_small_cases_every_element(w):
+    _full_case(w)
+
+
+def test_base_workload_every_element():
+    _full_case(workloads.BASE)
+
+
+@pytest.mark.parametrize("w", [workloads.QA, workloads.DILATED, workloads.LARGE], ids=lambda w: w.name)
+def test_full_size_workloads_sampled_rows(w):
+    inp = workloads.make_inputs(w)
+    got = parity.run_gpu(w, inp)
+    rows = parity.sample_rows(w, inp)
+    ref = parity.oracle_rows(w, inp, rows)
+    sel = got[rows[:, 0].tolist(), rows[:, 1].tolist(), rows[:, 2].tolist()]
+    parity.compare(w, sel, ref)
+    assert torch.isfinite(got.float()).all()
+
+
+EDGES = [
+    workloads.custom("T_lt_w", "bf16", 1, 2, 50, 64, 256, globals_per_b=[[3]], seed=21),
+    workloads.custom("r0", "bf16", 1, 2, 300, 64, 0, seed=22),
+    workloads.custom("r0_f32", "f32", 1, 2, 100, 16, 0, globals_per_b=[[9]], seed=23),
+    workloads.custom("no_globals", "bf16", 2, 2, 400, 64, 33, dil=[1, 2], seed=24),
+    workloads.custom("global_last", "bf16", 1, 2, 260, 64, 17, globals_per_b=[[259]], seed=25),
+    workloads.custom("padded_global", "bf16", 2, 2, 333, 64, 40, globals_per_b=[[300, 5], [320, 320]],
+                     pad_from=[290, 100], seed=26),
+    workloads.custom("all_padded_sample", "bf16", 2, 1, 256, 64, 30, globals_per_b=[[0], [1]],
+                     pad_from=[0, None], seed=27),
+    workloads.custom("all_padded_f32", "f32", 2, 1, 64, 16, 5, globals_per_b=[[0], [1]],
+                     pad_from=[0, None], seed=28),
+    workloads.custom("T_mod_dil", "bf16", 1, 3, 257, 64, 12, dil=[2, 3, 4], globals_per_b=[[256]], seed=29),
+    workloads.custom("T1", "bf16", 1, 1, 1, 64, 3, seed=30),
+    workloads.custom("T1_f32", "f32", 1, 1, 1, 8, 3, globals_per_b=[[0]], seed=31),
+    workloads.custom("T_129", "bf16", 1, 1, 129, 64, 128, globals_per_b=[[128, 128, 0]], seed=32),
+    workloads.custom("huge_r", "bf16", 1, 2, 400, 64, 100000, dil=[1, 3], seed=33),
+    workloads.custom("scale_2", "bf16", 1, 2, 300, 64, 50, globals_per_b=[[10]], scale=0.5, seed=34),
+]
+
+
+@pytest.mark.parametrize("w", EDGES, ids=lambda w: w.name)
+def test_edge_cases_every_element(w):
+    _full_case(w)
+
+
+def test_out_of_range_global_entries_are_ignored_and_flagged():
+    w = workloads.custom("bad_g", "bf16", 1, 2, 300, 64, 20, seed=40)
+    inp = workloads.make_inputs(w)
+    lf_attn.device_status()  # clear
+    inp["global_idx"] = torch.tensor([[-5, 7, 300, 7]], dtype=torch.int32)
+    got = parity.run_gpu(w, inp)
+    st, flags = lf_attn.device_status()
+    assert st == 5 and flags & 1
+    inp_ok = dict(inp)
+    inp_ok["global_idx"] = torch.tensor([[7]], dtype=torch.int32)
+    ref = parity.oracle_full(w, inp_ok)
+    parity.compare(w, got, ref)
+    st, flags = lf_attn.device_status()
+    assert st == 0 and flags == 0
+
+
+def test_deterministic_and_three_launches():
+    w = workloads.BASE
+    inp = workloads.make_inputs(w)
+    a = parity.run_gpu(w, inp)
+    assert lf_attn.last_launch_count() == 3
+    b = parity.run_gpu(w, inp)
+    assert torch.equal(a, b)
+
+
+def test_output_guard_regions_untouched():
+    w = workloads.custom("guard", "bf16", 1, 2, 333, 64, 40, globals_per_b=[[1, 200]], seed=41)
+    inp = workloads.make_inputs(w)
+    q, k, v = (inp[x].cuda() for x in ("q", "k", "v"))
+    n = q.numel()
+    guard = 4096
+    buf = torch.full((n + 2 * guard,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[guard:guard + n].view(q.shape)
+    lf_attn.fwd(q, k, v, w.r, dil=inp["dil"], global_idx=inp["global_idx"].cuda(), out=out,
+                scale=w.softmax_scale)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + n:] == 7.0)
+    parity.compare(w, out, parity.oracle_full(w, inp))
+
+
+def test_host_entry_point_matches_device_entry_point():
+    w = workloads.custom("host_api", "bf16", 2, 2, 700, 64, 60, globals_per_b=[[0, 5], [9, 9]],
+                         pad_from=[None, 600], seed=42)
+    inp = workloads.make_inputs(w)
+    dev = parity.run_gpu(w, inp)
+    pinned = {k: (v.pin_memory() if isinstance(v, torch.Tensor) and k != "dil" else v) for k, v in inp.items()}
+    host = lf_attn.fwd_host(pinned["q"], pinned["k"], pinned["v"], w.r, dil=inp["dil"],
+                            global_idx=pinned["global_idx"], key_pad_mask=pinned["key_pad_mask"],
+                            scale=w.softmax_scale)
+    assert torch.equal(host, dev.cpu())
+
+
+def test_argument_errors_on_gpu_do_not_launch():
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lf_attn.LfAttnError) as e:
+        lf_attn.fwd(q, q, q, -1)
+    assert e.value.status == 1
+    q32 = torch.zeros(1, 2, 64, 32, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lf_attn.LfAttnError) as e:
+        lf_attn.fwd(q32, q32, q32, 4)
+    assert e.value.status == 2
+    st, flags = lf_attn.device_status()
+    assert st == 0 and flags == 0
