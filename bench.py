@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sparse_long_sequence_fwd_b200 import flops as flops_mod  # noqa: E402
-from sparse_long_sequence_fwd_b200 import workloads  # noqa: E402
+from sparse_long_sequence_fwd_b200 import sharding, workloads  # noqa: E402
 
 METRIC = "useful sparse-attn TFLOP/s & tokens/s at T=4096,w=513; % of bf16 TC peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -276,11 +276,7 @@ def run_ours(args):
     t_wall1 = time.time()
     if world > 1:
         dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = sharding.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
     ms_per_step = ms / K
 
     # ---- per-kernel durations (each kernel alone, graph-replayed over the same rotating sets)
@@ -343,13 +339,9 @@ def run_ours(args):
                                  scale=w.softmax_scale, out=hout, stream=stream)
             b.record()
         torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = sharding.max_over_ranks(a.elapsed_time(b) / args.e2e_steps, device=dev)
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + tuple(x for x in (hg, hp) if x is not None))
-        e2e = {"value": round(world * total_f / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+        e2e = {"value": round(sharding.job_rate(total_f, world, e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(hout.numel() * hout.element_size()),
                "api": "lf_attn_fwd_host (pinned host buffers, copies inside the timed region)"}
@@ -358,8 +350,8 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, args.cpu_seconds)
 
-    tflops = world * total_f / (ms_per_step * 1e-3) / 1e12
-    tokens = world * w.B * w.T / (ms_per_step * 1e-3)
+    tflops = sharding.job_rate(total_f, world, ms_per_step * 1e-3) / 1e12
+    tokens = sharding.job_rate(w.B * w.T, world, ms_per_step * 1e-3)
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(tflops, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
@@ -406,17 +398,23 @@ def oracle_sample_rate(w, inp, seconds, seed=0):
         return np.stack([rng.integers(0, w.B, n), rng.integers(0, w.H, n), rng.integers(0, w.T, n)], 1).astype(
             np.int32)
 
-    probe = draw(64)
-    t0 = time.perf_counter()
-    oracle.rows(inp["q"], inp["k"], inp["v"], w.r, probe, dil=inp["dil"], global_idx=G, key_pad_mask=pad,
-                scale=w.softmax_scale)
-    dt = max(time.perf_counter() - t0, 1e-4)
-    n = int(min(max(64, 64 * seconds / dt), w.B * w.H * w.T))
+    def run(rows):
+        t0 = time.perf_counter()
+        oracle.rows(inp["q"], inp["k"], inp["v"], w.r, rows, dil=inp["dil"], global_idx=G, key_pad_mask=pad,
+                    scale=w.softmax_scale)
+        return time.perf_counter() - t0
+
+    # calibrate: grow the probe until it runs long enough to measure the rate
+    n = 256
+    while True:
+        dt = run(draw(n))
+        if dt >= min(0.5, seconds / 8) or n >= 64 * w.B * w.H * w.T:
+            break
+        n *= 4
+    # rows are drawn with replacement, so a cheap workload is sampled several times over
+    n = int(min(max(256, n * seconds / max(dt, 1e-4)), 64 * w.B * w.H * w.T))
     rows = draw(n)
-    t0 = time.perf_counter()
-    oracle.rows(inp["q"], inp["k"], inp["v"], w.r, rows, dil=inp["dil"], global_idx=G, key_pad_mask=pad,
-                scale=w.softmax_scale)
-    dt = time.perf_counter() - t0
+    dt = run(rows)
     return row_flops(rows.tolist()), dt, n, oracle.max_threads()
 
 
