@@ -51,7 +51,8 @@ typedef enum {
     LF_ERR_UNSUPPORTED = 2,  /* valid but outside what this build implements (see lf_attn_fwd) */
     LF_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed */
     LF_ERR_NO_MEMORY = 4,    /* workspace could not be allocated (or not during capture) */
-    LF_ERR_DEVICE_CHECK = 5  /* a device-side check fired (see lf_attn_device_status) */
+    LF_ERR_DEVICE_CHECK = 5, /* a device-side check fired (see lf_attn_device_status) */
+    LF_ERR_SCRATCH_TOO_SMALL = 6 /* lf_attn_fwd_static: sizes need more than its fixed scratch */
 } lf_status;
 
 /*
@@ -134,6 +135,41 @@ uint64_t lf_attn_workspace_bytes(int B, int H, int T, int d, int n_global, lf_dt
 
 /* Kernels launched by the last successful lf_attn_fwd on this host thread. */
 int lf_attn_last_launch_count(void);
+
+/*
+ * lf_attn_fwd_static -- lf_attn_fwd for callers that cannot allocate device
+ * memory (the pages describe no counterpart; this is a deployment variant).
+ *
+ * Some callers cannot call cudaMalloc: code running while a CUDA graph is
+ * captured in global mode, processes confined to a fixed memory budget or
+ * to their own pool allocator, runtimes that reserve all device memory at
+ * start-up.  This entry point allocates nothing, neither itself nor through
+ * any library: its workspace is a fixed scratch array compiled into this
+ * library (one per GPU that loads the library, 32 MiB minus a 256-byte
+ * status word, held until the process exits).
+ *
+ *   Arguments, layouts, ownership and the result are those of lf_attn_fwd;
+ *   the caller still provides q, k, v, out, global_idx and key_pad_mask.
+ *   Returns LF_ERR_SCRATCH_TOO_SMALL, before launching anything, when these
+ *   sizes need more than 32 MiB - 256 bytes of workspace (the
+ *   lf_attn_workspace_bytes figure); the five reference workloads need at
+ *   most about 9 MiB.
+ *   The first call on a device sets that device up (kernel attributes and
+ *   the scratch array's device address); make that first call before any
+ *   stream capture.
+ *   Every call on a device shares the one scratch array, which keeps the
+ *   last call's contents (the prep kernel clears what must start at zero).
+ *   Calls whose kernels overlap on the GPU -- on different streams, or
+ *   concurrently with another host thread -- race on that array.
+ *   Device-side flags of this variant (out-of-range global_idx entries,
+ *   which are ignored as in lf_attn_fwd; a pipeline wait that gave up) stay
+ *   in its scratch area and are not reported: check global_idx on the host.
+ */
+lf_status lf_attn_fwd_static(const void* q, const void* k, const void* v, void* out,
+                             int B, int H, int T, int d, int r, const int32_t* dil,
+                             const int32_t* global_idx, int n_global,
+                             const uint8_t* key_pad_mask, float scale, lf_dtype dtype,
+                             void* stream);
 
 #ifdef __cplusplus
 }

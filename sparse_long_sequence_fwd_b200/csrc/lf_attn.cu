@@ -355,6 +355,60 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
     return LF_OK;
 }
 
+// ------------------------------------------------------------------------
+// Allocation-free variant.  Some callers cannot call cudaMalloc at all: code
+// that runs while a CUDA graph is being captured in global mode, processes
+// under a strict memory budget or a custom pool that forbids the runtime's
+// allocator, or embedded runtimes that reserve all device memory up front.
+// For them lf_attn_fwd_static runs the same kernels on a fixed scratch area
+// that the module image carries: one file-scope __device__ array per GPU that
+// loads this library, held until the process exits.  Its first 256 bytes
+// take the device-side flags of this variant; the rest is the workspace.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+struct StaticState {
+    bool init = false;
+    int sm_count = 0;
+    uint8_t* scratch = nullptr;  // device address of g_static_scratch on this device
+};
+StaticState g_static[kMaxDevices];
+
+// Once per device, with that device current: kernel attributes and the
+// device address of the scratch array (the host-side symbol is only a
+// stand-in and must never reach a kernel).  Allocates nothing.
+lf_status static_state(StaticState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_CUDA;
+    StaticState& s = g_static[dev];
+    if (!s.init) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LF_ERR_CUDA;
+        if (prop.major < 10) return LF_ERR_UNSUPPORTED;
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return LF_ERR_CUDA;
+        const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + kMaxGlobal) * 4;
+        const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
+        if (cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) != cudaSuccess ||
+            cudaFuncSetAttribute(global_rows_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gr_max) != cudaSuccess ||
+            cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gr_max) != cudaSuccess ||
+            cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gr_max) != cudaSuccess ||
+            cudaFuncSetAttribute(global_rows_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGrBf16Smem) != cudaSuccess)
+            return LF_ERR_CUDA;
+        s.sm_count = prop.multiProcessorCount;
+        s.scratch = static_cast<uint8_t*>(ptr);
+        s.init = true;
+    }
+    *out = &s;
+    return LF_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -444,6 +498,8 @@ const char* lf_attn_strerror(lf_status s) {
         case LF_ERR_CUDA: return "CUDA error";
         case LF_ERR_NO_MEMORY: return "workspace allocation failed (or attempted during stream capture)";
         case LF_ERR_DEVICE_CHECK: return "device-side check failed";
+        case LF_ERR_SCRATCH_TOO_SMALL:
+            return "the workspace these sizes need exceeds the static scratch of lf_attn_fwd_static (32 MiB)";
     }
     return "unknown status";
 }
@@ -470,5 +526,29 @@ uint64_t lf_attn_workspace_bytes(int B, int H, int T, int d, int n_global, lf_dt
 }
 
 int lf_attn_last_launch_count(void) { return t_last_launches; }
+
+lf_status lf_attn_fwd_static(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d,
+                             int r, const int32_t* dil, const int32_t* global_idx, int n_global,
+                             const uint8_t* key_pad_mask, float scale, lf_dtype dtype, void* stream) {
+    lf_status st = check_args(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, scale, dtype);
+    if (st != LF_OK) return st;
+    const size_t cap = kStaticScratchBytes - 256;
+    if (make_layout(B, H, T, d, n_global, dtype).total > cap) return LF_ERR_SCRATCH_TOO_SMALL;
+    std::lock_guard<std::mutex> lock(g_mu);
+    StaticState* ss = nullptr;
+    if ((st = static_state(&ss)) != LF_OK) return st;
+    // The workspace already has the capacity the layout needs, so launch_all
+    // never grows (allocates) it.  Prep zeroes what must start at zero.
+    DeviceState view;
+    view.init = true;
+    view.sm_count = ss->sm_count;
+    view.status = reinterpret_cast<uint32_t*>(ss->scratch);
+    view.ws = ss->scratch + 256;
+    view.ws_bytes = cap;
+    return launch_all(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, key_pad_mask, scale, dtype,
+                      static_cast<cudaStream_t>(stream), &view);
+}
+
+
 
 }  // extern "C"

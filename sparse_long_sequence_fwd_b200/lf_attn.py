@@ -17,9 +17,10 @@ LIB_PATH = os.path.join(_PKG, "liblfattn.so")
 
 LF_F32, LF_BF16 = 0, 1
 STATUS = {0: "LF_OK", 1: "LF_ERR_INVALID_ARG", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
-          4: "LF_ERR_NO_MEMORY", 5: "LF_ERR_DEVICE_CHECK"}
+          4: "LF_ERR_NO_MEMORY", 5: "LF_ERR_DEVICE_CHECK", 6: "LF_ERR_SCRATCH_TOO_SMALL"}
 EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
-           "lf_attn_release", "lf_attn_workspace_bytes", "lf_attn_last_launch_count")
+           "lf_attn_release", "lf_attn_workspace_bytes", "lf_attn_last_launch_count",
+           "lf_attn_fwd_static")
 
 _lib = None
 
@@ -55,6 +56,9 @@ def load():
         lib.lf_attn_workspace_bytes.restype = ctypes.c_uint64
         lib.lf_attn_last_launch_count.argtypes = []
         lib.lf_attn_last_launch_count.restype = I
+        lib.lf_attn_fwd_static.argtypes = sig
+        lib.lf_attn_fwd_static.restype = I
+
         _lib = lib
     return _lib
 
@@ -154,6 +158,32 @@ def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, r: int, dil=None
                                  ctypes.c_void_p(s.cuda_stream))
     if st != 0:
         raise LfAttnError(st, "lf_attn_fwd_host")
+    return out
+
+
+def fwd_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, r: int, dil=None,
+               global_idx: Optional[torch.Tensor] = None, key_pad_mask: Optional[torch.Tensor] = None,
+               scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """lf_attn_fwd_static on CUDA tensors: the forward on the library's fixed
+    32 MiB scratch array, for callers that cannot allocate device memory
+    (graph capture in global mode, fixed budgets, own pool allocators).  Such
+    callers pass ``out`` in (otherwise torch allocates it here)."""
+    _check_qkv(q, k, v)
+    B, H, T, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    n_global = 0 if global_idx is None else global_idx.shape[1]
+    if n_global == 0:
+        global_idx = None
+    if scale is None:
+        scale = d ** -0.5
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = load().lf_attn_fwd_static(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, d, int(r), _dil_array(dil, H),
+                                   _ptr(global_idx), n_global, _ptr(key_pad_mask), float(scale), _dtype_code(q),
+                                   ctypes.c_void_p(s.cuda_stream))
+    if st != 0:
+        raise LfAttnError(st, "lf_attn_fwd_static")
     return out
 
 
