@@ -17,13 +17,20 @@
 //                                   count rounded to 16), K=64 -> TMEM (fp32),
 //                                   double-buffered so the next block's S is
 //                                   computed during this block's softmax
-//                  online softmax   two threads per query row (64 columns
-//                                   each): mask, row max (the two halves
-//                                   swap partial maxima through shared
-//                                   memory), exp2, partial row sums, fp32
-//                  O += P V         P (bf16) through 128B-swizzled shared
-//                                   memory, tcgen05.mma M=128, N=64; the
-//                                   accumulator O stays in TMEM
+//                  online softmax   two threads per query row, one per half
+//                                   of the block's 128 key columns; each
+//                                   keeps its own running max and exponent
+//                                   base (fp32, log2 domain)
+//                  O_h += P_h V_h   P (bf16) through 128B-swizzled shared
+//                                   memory (double-buffered); the PV
+//                                   product's first 4 k-steps (keys 0..63)
+//                                   accumulate into O_0, the last 4 into
+//                                   O_1, so each half's exponent base
+//                                   stays private; M=128, N=64, in TMEM
+//                  L_h += P_h 1     row sums from the tensor core too (N=16
+//                                   against a tile of ones)
+// At the end of a tile the two halves swap bases once and each writes half
+// of the output row: y = (2^m0 O_0 + 2^m1 O_1) / (2^m0 L_0 + 2^m1 L_1).
 // The exponent base of a row is only moved (and O, l rescaled in place) when
 // the running max exceeds it by more than 2^8; otherwise p = 2^(s - base)
 // stays below 256, which fp32 accumulation and bf16 P absorb exactly as well.
@@ -36,7 +43,9 @@
 // issuer (warp 1 also owns the TMEM allocation), warps 2..5 softmax of key
 // columns 0..63, warps 6..9 softmax of columns 64..127 of the same rows (warp
 // w serves TMEM lanes 32*(w%4)..+31).  Every hand-off is an mbarrier and
-// every wait is bounded (ptx.cuh).
+// every wait is bounded (ptx.cuh).  In steady state the softmax warps never
+// wait on a round trip through the MMA warp: S is double-buffered, and P(k)
+// only needs the product of block k-2 to have finished.
 #pragma once
 #include "lf_common.cuh"
 #include "ptx.cuh"
@@ -46,7 +55,7 @@ namespace lf {
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kHD = 64;
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 constexpr int kTileBytes = kBM * kHD * 2;  // 16 KB: 128 rows x 128 bytes
 constexpr int kBandThreads = 320;
 constexpr int kSoftmaxWarp0 = 2;           // warps 2..9
@@ -55,13 +64,14 @@ constexpr float kRescaleLog2 = 8.f;        // move the exponent base only past 2
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kTileBytes;                  // kStages x 16 KB
 constexpr int kOffV = kOffK + kStages * kTileBytes;        // kStages x 16 KB
-constexpr int kOffP = kOffV + kStages * kTileBytes;        // 2 x 16 KB (keys 0..63 | 64..127)
-constexpr int kOffX = kOffP + 2 * kTileBytes;              // row-max exchange: [2 parity][2 half][128] f32
+constexpr int kOffP = kOffV + kStages * kTileBytes;        // 2 buffers x (keys 0..63 | 64..127) x 16 KB
+constexpr int kOffOnes = kOffP + 2 * 2 * kTileBytes;       // 16 x 128 bf16 ones (row-sum operand), 4 KB
+constexpr int kOffX = kOffOnes + 4096;                     // per-tile exchange of bases: [2 parity][2 half][128] f32
 constexpr int kOffBar = kOffX + 2 * 2 * kBM * 4;
 // barrier slots
 constexpr int kBarQFull = 0, kBarQEmpty = 1, kBarKvFull = 2, kBarKvEmpty = kBarKvFull + kStages,
               kBarSFull = kBarKvEmpty + kStages, kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2,
-              kBarOFull = kBarPFull + 1, kBarXchg = kBarOFull + 1, kBarDrain = kBarXchg + 4,
+              kBarOFull = kBarPFull + 2, kBarXchg = kBarOFull + 2, kBarDrain = kBarXchg + 4,
               kNumBars = kBarDrain + 1;
 constexpr int kOffMisc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
 constexpr int kMiscBytes = 16;
@@ -69,9 +79,13 @@ constexpr int kBandSmem = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 static_assert(kBandSmem <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S buffers at 0 and 128 (fp32, 128 wide), O at 256 (fp32, 64 wide)
+// TMEM columns: S buffers at 0 and 128 (fp32, 128 wide); per key half h
+// (keys 0..63 / 64..127 of every block) an output accumulator O_h at
+// 256 + 64 h (fp32, 64 wide) and a row-sum accumulator L_h at 384 + 16 h
+// (fp32, 16 identical columns: P times a ones tile).
 __device__ __forceinline__ uint32_t col_s(uint32_t buf) { return buf * 128u; }
-constexpr uint32_t kColO = 256u;
+__device__ __forceinline__ uint32_t col_o(uint32_t h) { return 256u + 64u * h; }
+__device__ __forceinline__ uint32_t col_l(uint32_t h) { return 384u + 16u * h; }
 
 struct BandTile {
     int b, bh, c, dil, dk, R;
@@ -126,9 +140,36 @@ __device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
 }
 
 // ------------------------------------------------------------ softmax role
-// Thread (row x, half hf) owns key columns [64 hf, 64 hf + 64) of row x.
-// POS: scale > 0, so maxima are taken on raw scores and the scale is folded
-// into the exp2 argument.
+// Thread (row x, half hf) owns key columns [64 hf, 64 hf + 64) of row x but
+// reads all 128 for the row max.  POS: scale > 0, so maxima are taken on raw
+// scores and the scale is folded into the exp2 argument.
+template <bool POS, bool KEEP = true>
+__device__ __forceinline__ float masked_max32(uint32_t* v, uint32_t mk, bool full, float sl2) {
+    float mxp[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) mxp[u] = -INFINITY;
+    if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            float f = __uint_as_float(v[j]);
+            if (!POS) f *= sl2;
+            if (KEEP) v[j] = __float_as_uint(f);
+            mxp[j & 7] = fmaxf(mxp[j & 7], f);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            float f = __uint_as_float(v[j]);
+            if (!POS) f *= sl2;
+            f = ((mk >> j) & 1u) ? f : -INFINITY;
+            if (KEEP) v[j] = __float_as_uint(f);
+            mxp[j & 7] = fmaxf(mxp[j & 7], f);
+        }
+    }
+    return fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                 fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+}
+
 template <bool POS>
 __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                              volatile int* abort_flag, uint32_t tmem_base) {
@@ -137,13 +178,14 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     const int hf = (warp - kSoftmaxWarp0) >> 2;  // column half
     const int x = wq * 32 + lane;                // query row inside the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tO = tmem_base + lane_off + kColO + 32u * hf;  // this half of the output row
-    uint8_t* pbuf = smem + kOffP + hf * kTileBytes;               // P keys [64 hf, 64 hf + 64)
-    float* xm = reinterpret_cast<float*>(smem + kOffX);           // [2 parity][2 half][128]
+    const uint32_t tO = tmem_base + lane_off + col_o(hf);  // this key half's output accumulator
+    const uint32_t tL = tmem_base + lane_off + col_l(hf);  // ... and row-sum accumulator
+    float* xm = reinterpret_cast<float*>(smem + kOffX);    // [2 parity][2 half][128]
     uint64_t* xbar = &bars[kBarXchg + wq];
+    uint32_t x_cnt = 0;
     const int rowoff = (x >> 3) * 1024 + (x & 7) * 128;
     const float sl2 = p.sl2;
-    uint32_t blk_it = 0, pv_cnt = 0, x_cnt = 0;
+    uint32_t blk_it = 0;  // key blocks processed by this CTA (all tiles)
 
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
         int ok = 1;
@@ -152,6 +194,8 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
         __syncwarp();  // memory order for the other lanes
         return ok != 0;
     };
+    // block j's product O += P V has completed (barrier of P buffer j % 2)
+    auto wait_pv = [&](uint32_t j) -> bool { return wait_warp(&bars[kBarOFull + (j & 1u)], (j >> 1) & 1u); };
     // swap one float per row with the other half's thread of the same row
     auto exchange = [&](float mine, float* other) -> bool {
         float* slot = xm + (x_cnt & 1u) * (2 * kBM);
@@ -175,12 +219,11 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
 
         float m_run = -INFINITY;  // running row max (scaled, log2 domain)
         float m_ref = -INFINITY;  // exponent base in use (-inf: nothing valid yet)
-        float l_half = 0.f;       // this half's share of the row sum
         const int nb = t.nbb + t.ngb;
         for (int blk = 0; blk < nb; ++blk, ++blk_it) {
             const uint32_t sb = blk_it & 1u;
             const bool band = blk < t.nbb;
-            uint32_t mk[2];
+            uint32_t mk[2];  // valid-key bits of this half's two 32-column chunks
             uint32_t need = 0;
             int ncols = kBN;
             if (band) {
@@ -224,107 +267,79 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                     }
                 }
             }
+            bool full[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) full[u] = __all_sync(0xffffffffu, mk[u] == 0xffffffffu);
 
-            // ---- this half of the S block from TMEM
+            // ---- this half's 64 columns of the S block
             if (!wait_warp(&bars[kBarSFull + sb], (blk_it >> 1) & 1u)) return;
             tc_fence_after();
-            uint32_t sr[64];
             const uint32_t tS = tmem_base + lane_off + col_s(sb) + 64u * hf;
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-                if (need & (1u << u)) tmem_ld32(tS + 32 * u, sr + 32 * u);
+            uint32_t sr[64];
+            if (need & 1u) tmem_ld32(tS, sr);
+            if (need & 2u) tmem_ld32(tS + 32, sr + 32);
             tmem_ld_wait(sr);
             reg_fence32(sr + 32);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[kBarSFree + sb]);
 
-            // ---- mask and partial row max (8 independent chains)
-            float mxp[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) mxp[u] = -INFINITY;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (need & (1u << u)) {
-                    if (__all_sync(0xffffffffu, mk[u] == 0xffffffffu)) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            float v = __uint_as_float(sr[32 * u + j]);
-                            if (!POS) v *= sl2;
-                            sr[32 * u + j] = __float_as_uint(v);
-                            mxp[j & 7] = fmaxf(mxp[j & 7], v);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            float v = __uint_as_float(sr[32 * u + j]);
-                            if (!POS) v *= sl2;
-                            v = ((mk[u] >> j) & 1u) ? v : -INFINITY;
-                            sr[32 * u + j] = __float_as_uint(v);
-                            mxp[j & 7] = fmaxf(mxp[j & 7], v);
-                        }
-                    }
-                }
-            }
-            float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+            float mx = -INFINITY;
+            if (need & 1u) mx = masked_max32<POS>(sr, mk[0], full[0], sl2);
+            if (need & 2u) mx = fmaxf(mx, masked_max32<POS>(sr + 32, mk[1], full[1], sl2));
             if (POS) mx *= sl2;  // -inf stays -inf
-            float mx_other;
-            if (!exchange(mx, &mx_other)) return;
-            m_run = fmaxf(m_run, fmaxf(mx, mx_other));
+            m_run = fmaxf(m_run, mx);
 
-            // ---- P buffer and O are free once the previous block's PV has completed
-            if (blk > 0 && !wait_warp(&bars[kBarOFull], (pv_cnt - 1) & 1u)) return;
-            // ---- move the exponent base if the max ran past it (rare): rescale O and l
+            // ---- move this half's exponent base if its max ran past it (rare): rescale O_h and L_h
             float alpha = 1.f;
             bool move = (m_run != -INFINITY) && (m_ref == -INFINITY || m_run > m_ref + kRescaleLog2);
             if (blk == 0) {
-                m_ref = m_run;  // the first PV overwrites O
+                m_ref = m_run;  // the first product of the tile overwrites O_h and L_h
                 move = false;
             } else if (move) {
                 alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_run);
                 m_ref = m_run;
-                l_half *= alpha;
             }
             if (__any_sync(0xffffffffu, move)) {
+                if (!wait_pv(blk_it - 1)) return;  // O_h and L_h hold every earlier product
                 tc_fence_after();
                 uint32_t orr[32];
-                tmem_ld32(tO, orr);
-                tmem_ld_wait(orr);
+#pragma unroll 1
+                for (int part = 0; part < 2; ++part) {  // O_h, 32 columns at a time
+                    tmem_ld32(tO + 32u * part, orr);
+                    tmem_ld_wait(orr);
 #pragma unroll
-                for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-                tmem_st32(tO, orr);
+                    for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+                    tmem_st32(tO + 32u * part, orr);
+                }
+                tmem_ld16(tL, orr);  // L_h: exactly its 16 columns
+                tmem_ld_wait16(orr);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+                tmem_st16(tL, orr);
                 tmem_st_wait();
             }
             const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
 
-            // ---- p = 2^(s - base), partial row sum, P (bf16) into the 128B-swizzled K-major buffer
-            float rsp[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) rsp[u] = 0.f;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (need & (1u << u)) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float v = __uint_as_float(sr[32 * u + j]);
-                        const float e = POS ? ex2_approx(fmaf(v, sl2, -base)) : ex2_approx(v - base);
-                        sr[32 * u + j] = __float_as_uint(e);
-                        rsp[j & 7] += e;
-                    }
-                }
-            }
-            l_half += ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7]));
+            // ---- p = 2^(s - base) on this half, as bf16 into P buffer sb once the
+            //      product of block blk_it - 2 has read that buffer
+            if (blk_it >= 2 && !wait_pv(blk_it - 2)) return;
+            uint8_t* pbuf = smem + kOffP + sb * (2 * kTileBytes) + hf * kTileBytes;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
                 if (64 * hf + 8 * ch < ncols) {
                     uint4 val = make_uint4(0u, 0u, 0u, 0u);
                     if (need & (1u << (ch >> 2))) {
-                        const uint32_t* e = sr + 8 * ch;
-                        val.x = pack_bf16x2(__uint_as_float(e[0]), __uint_as_float(e[1]));
-                        val.y = pack_bf16x2(__uint_as_float(e[2]), __uint_as_float(e[3]));
-                        val.z = pack_bf16x2(__uint_as_float(e[4]), __uint_as_float(e[5]));
-                        val.w = pack_bf16x2(__uint_as_float(e[6]), __uint_as_float(e[7]));
+                        float e[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float v = __uint_as_float(sr[8 * ch + j]);
+                            e[j] = POS ? ex2_approx(fmaf(v, sl2, -base)) : ex2_approx(v - base);
+                        }
+                        val.x = pack_bf16x2(e[0], e[1]);
+                        val.y = pack_bf16x2(e[2], e[3]);
+                        val.z = pack_bf16x2(e[4], e[5]);
+                        val.w = pack_bf16x2(e[6], e[7]);
                     }
                     *reinterpret_cast<uint4*>(pbuf + rowoff + ((ch ^ (x & 7)) << 4)) = val;
                 }
@@ -332,34 +347,56 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kBarPFull]);
-            ++pv_cnt;
+            if (lane == 0) mbar_arrive(&bars[kBarPFull + sb]);
         }
 
-        // ---- epilogue: this half of O / l (global rows are written by K2)
-        float l_other;
-        if (!exchange(l_half, &l_other)) return;
-        if (!wait_warp(&bars[kBarOFull], (pv_cnt - 1) & 1u)) return;
+        // ---- epilogue: output columns [32 hf, 32 hf + 32) of this row from both key
+        //      halves, y = (2^m0 O_0 + 2^m1 O_1) / (2^m0 L_0 + 2^m1 L_1)
+        //      (global rows are written by K2)
+        float m_other;
+        if (!exchange(m_ref, &m_other)) return;
+        if (!wait_pv(blk_it - 1)) return;
         tc_fence_after();
-        uint32_t o[32];
-        tmem_ld32(tO, o);
-        tmem_ld_wait(o);
-        tc_fence_before();
-        if (row_ok) {
-            const float l = l_half + l_other;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t.bh) * p.T + i) * kHD + 32 * hf);
+        const float m0 = hf == 0 ? m_ref : m_other, m1 = hf == 0 ? m_other : m_ref;
+        const float mm = fmaxf(m0, m1);
+        const float f0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - mm);
+        const float f1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - mm);
+        float l0, l1;
+        {
+            uint32_t lr[16];
+            tmem_ld16(tmem_base + lane_off + col_l(0), lr);
+            tmem_ld_wait16(lr);
+            l0 = __uint_as_float(lr[0]);
+            tmem_ld16(tmem_base + lane_off + col_l(1), lr);
+            tmem_ld_wait16(lr);
+            l1 = __uint_as_float(lr[0]);
+        }
+        const float l = f0 * l0 + f1 * l1;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t.bh) * p.T + i) * kHD + 32 * hf);
+#pragma unroll 1
+        for (int q16 = 0; q16 < 2; ++q16) {  // 16 output columns at a time
+            uint32_t a0[16], a1[16];
+            tmem_ld16(tmem_base + lane_off + col_o(0) + 32u * hf + 16u * q16, a0);
+            tmem_ld16(tmem_base + lane_off + col_o(1) + 32u * hf + 16u * q16, a1);
+            tmem_ld_wait16(a0);
+            reg_fence16(a1);
+            float y[16];
 #pragma unroll
-            for (int v8 = 0; v8 < 4; ++v8) {
-                const uint32_t* src = o + 8 * v8;
-                uint4 val;
-                val.x = pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
-                val.y = pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
-                val.z = pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
-                val.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
-                dst[v8] = val;
+            for (int c = 0; c < 16; ++c) y[c] = (f0 * __uint_as_float(a0[c]) + f1 * __uint_as_float(a1[c])) * inv;
+            if (row_ok) {
+#pragma unroll
+                for (int v8 = 0; v8 < 2; ++v8) {
+                    uint4 val;
+                    val.x = pack_bf16x2(y[8 * v8 + 0], y[8 * v8 + 1]);
+                    val.y = pack_bf16x2(y[8 * v8 + 2], y[8 * v8 + 3]);
+                    val.z = pack_bf16x2(y[8 * v8 + 4], y[8 * v8 + 5]);
+                    val.w = pack_bf16x2(y[8 * v8 + 6], y[8 * v8 + 7]);
+                    dst[2 * q16 + v8] = val;
+                }
             }
         }
+        tc_fence_before();
     }
 }
 
@@ -385,8 +422,10 @@ __global__ void __launch_bounds__(kBandThreads, 1) band_tc_kernel(const __grid_c
             mbar_init(&bars[kBarSFull + s], 1);
             mbar_init(&bars[kBarSFree + s], 8);
         }
-        mbar_init(&bars[kBarPFull], 8);
-        mbar_init(&bars[kBarOFull], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[kBarPFull + s], 8);
+            mbar_init(&bars[kBarOFull + s], 1);
+        }
         for (int w = 0; w < 4; ++w) mbar_init(&bars[kBarXchg + w], 2);
         mbar_init(&bars[kBarDrain], 1);
         *abort_flag = 0;
@@ -404,6 +443,11 @@ __global__ void __launch_bounds__(kBandThreads, 1) band_tc_kernel(const __grid_c
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
+    }
+    {  // the ones tile (bf16 1.0) read by the row-sum MMA
+        uint32_t* ones = reinterpret_cast<uint32_t*>(smem + kOffOnes);
+        for (int u = threadIdx.x; u < 1024; u += kBandThreads) ones[u] = 0x3F803F80u;
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -462,20 +506,27 @@ __global__ void __launch_bounds__(kBandThreads, 1) band_tc_kernel(const __grid_c
             const uint32_t sK0 = smem_u32(smem + kOffK);
             const uint32_t sV0 = smem_u32(smem + kOffV);
             const uint32_t sP = smem_u32(smem + kOffP);
-            uint32_t kv_it = 0, q_it = 0, blk_it = 0, pv_it = 0;
+            const uint32_t idesc_l = idesc_bf16(kBM, 16, 0, 0);
+            const uint32_t sOnes = smem_u32(smem + kOffOnes);
+            uint32_t kv_it = 0, q_it = 0, blk_it = 0;
             bool alive = true;
-            auto issue_pv = [&](uint32_t stage, int nk, bool first) -> bool {
-                if (!mbar_wait(&bars[kBarPFull], pv_it & 1u, abort_flag)) return false;
+            // O += P V and l += P 1 for block j (P buffer j % 2)
+            auto issue_pv = [&](uint32_t j, uint32_t stage, int nk, bool first) -> bool {
+                const uint32_t pb = j & 1u;
+                if (!mbar_wait(&bars[kBarPFull + pb], (j >> 1) & 1u, abort_flag)) return false;
                 tc_fence_after();
+                const uint32_t aP = sP + pb * (2 * kTileBytes);
                 const uint32_t bV = sV0 + stage * kTileBytes;
                 for (int ks = 0; ks < nk / 16; ++ks) {
-                    const uint64_t ad = sdesc_k_sw128(sP + (ks >> 2) * kTileBytes + (ks & 3) * 32);
-                    const uint64_t bd = sdesc_mn_sw128(bV + ks * 2048);
-                    tc_mma_ss(tmem_base + kColO, ad, bd, idesc_pv, (ks > 0 || !first) ? 1u : 0u);
+                    // k-steps 0..3 cover keys 0..63 (accumulators of half 0), 4..7 keys 64..127 (half 1)
+                    const uint32_t h = static_cast<uint32_t>(ks >> 2);
+                    const uint64_t ad = sdesc_k_sw128(aP + h * kTileBytes + (ks & 3) * 32);
+                    const uint32_t acc = ((ks & 3) > 0 || !first) ? 1u : 0u;
+                    tc_mma_ss(tmem_base + col_o(h), ad, sdesc_mn_sw128(bV + ks * 2048), idesc_pv, acc);
+                    tc_mma_ss(tmem_base + col_l(h), ad, sdesc_k_sw128(sOnes + h * 2048 + (ks & 3) * 32), idesc_l, acc);
                 }
-                tc_commit(&bars[kBarOFull]);
+                tc_commit(&bars[kBarOFull + pb]);
                 tc_commit(&bars[kBarKvEmpty + stage]);
-                ++pv_it;
                 return true;
             };
             for (int item = blockIdx.x; item < p.n_items && alive; item += gridDim.x) {
@@ -504,7 +555,7 @@ __global__ void __launch_bounds__(kBandThreads, 1) band_tc_kernel(const __grid_c
                                   idesc_s, ks > 0 ? 1u : 0u);
                     tc_commit(&bars[kBarSFull + sb]);
                     if (blk == nb - 1) tc_commit(&bars[kBarQEmpty]);
-                    if (blk > 0 && !issue_pv(prev_stage, prev_nk, blk == 1)) {
+                    if (blk > 0 && !issue_pv(blk_it - 1, prev_stage, prev_nk, blk == 1)) {
                         alive = false;
                         break;
                     }
@@ -513,7 +564,7 @@ __global__ void __launch_bounds__(kBandThreads, 1) band_tc_kernel(const __grid_c
                     ++blk_it;
                     ++kv_it;
                 }
-                if (alive && !issue_pv(prev_stage, prev_nk, nb == 1)) alive = false;
+                if (alive && !issue_pv(blk_it - 1, prev_stage, prev_nk, nb == 1)) alive = false;
             }
             // all MMAs issued by this thread complete before TMEM is released
             tc_commit(&bars[kBarDrain]);

@@ -93,12 +93,27 @@ EDGES = [
     workloads.custom("T_129", "bf16", 1, 1, 129, 64, 128, globals_per_b=[[128, 128, 0]], seed=32),
     workloads.custom("huge_r", "bf16", 1, 2, 400, 64, 100000, dil=[1, 3], seed=33),
     workloads.custom("scale_2", "bf16", 1, 2, 300, 64, 50, globals_per_b=[[10]], scale=0.5, seed=34),
+    # large score spread: the running max moves past the exponent base often
+    workloads.custom("scale_big", "bf16", 1, 2, 900, 64, 256, globals_per_b=[[3, 700]], scale=2.0, seed=35),
+    workloads.custom("scale_big_f32", "f32", 1, 2, 300, 32, 40, globals_per_b=[[3]], scale=2.0, seed=36),
+    workloads.custom("scale_negative", "bf16", 1, 2, 400, 64, 60, globals_per_b=[[0]], scale=-0.3, seed=37),
 ]
 
 
 @pytest.mark.parametrize("w", EDGES, ids=lambda w: w.name)
 def test_edge_cases_every_element(w):
     _full_case(w)
+
+
+def test_growing_key_norms_move_the_exponent_base():
+    """Key norms grow along the sequence, so a row's max rises block after
+    block by far more than 2^8 and the band kernel rescales O and l in place
+    many times; the result must still match the oracle."""
+    w = workloads.custom("growing", "bf16", 1, 2, 1100, 64, 300, dil=[1, 2], globals_per_b=[[1000]], seed=38)
+    inp = workloads.make_inputs(w)
+    ramp = torch.linspace(0.2, 6.0, w.T).reshape(1, 1, w.T, 1)
+    inp["k"] = (inp["k"].float() * ramp).to(torch.bfloat16)
+    parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
 
 
 def test_out_of_range_global_entries_are_ignored_and_flagged():
