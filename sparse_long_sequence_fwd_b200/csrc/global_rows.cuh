@@ -61,6 +61,47 @@ __device__ __forceinline__ float block_reduce_sum(float v, float* red) {
     return r;
 }
 
+// Merge of the per-chunk partial states of every global query of one (b, h)
+// by the last CTA to arrive: M = max_c m_c, w_c = 2^(m_c - M),
+// y = sum_c w_c acc_c / sum_c w_c l_c.  Every load is independent of the
+// values loaded before it, so the partials stream in parallel.
+template <typename Tout>
+__device__ __forceinline__ void merge_partials(const GlobalRowParams& p, int bh, int nq, const int32_t* gq, int d) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int stride = d + 2;
+    for (int a = warp; a < nq; a += kGrThreads / 32) {
+        const float* src = p.ws.partial + (static_cast<size_t>(bh) * p.gstride + a) * p.nchunk * stride;
+        float M = -INFINITY;
+        for (int c = lane; c < p.nchunk; c += 32) M = fmaxf(M, __ldcg(src + static_cast<size_t>(c) * stride));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float Mu = (M == -INFINITY) ? 0.f : M;  // every chunk empty: all weights 0
+        float L = 0.f;
+        for (int c = lane; c < p.nchunk; c += 32)
+            L = fmaf(exp2f(__ldcg(src + static_cast<size_t>(c) * stride) - Mu),
+                     __ldcg(src + static_cast<size_t>(c) * stride + 1), L);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        Tout* orow = reinterpret_cast<Tout*>(p.out) + (static_cast<size_t>(bh) * p.T + gq[a]) * d;
+        for (int col = lane; col < d; col += 32) {
+            float acc0 = 0.f, acc1 = 0.f;
+            int c = 0;
+            for (; c + 1 < p.nchunk; c += 2) {
+                const float* p0 = src + static_cast<size_t>(c) * stride;
+                const float* p1 = p0 + stride;
+                acc0 = fmaf(exp2f(__ldcg(p0) - Mu), __ldcg(p0 + 2 + col), acc0);
+                acc1 = fmaf(exp2f(__ldcg(p1) - Mu), __ldcg(p1 + 2 + col), acc1);
+            }
+            if (c < p.nchunk) {
+                const float* p0 = src + static_cast<size_t>(c) * stride;
+                acc0 = fmaf(exp2f(__ldcg(p0) - Mu), __ldcg(p0 + 2 + col), acc0);
+            }
+            store_from_float(orow + col, (acc0 + acc1) * inv);
+        }
+    }
+}
+
 // DP: head dim rounded up to a multiple of 32 (32, 64 or 128).
 template <typename Tin, int DP>
 __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams p) {
@@ -142,31 +183,7 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int a = warp; a < nq; a += kGrThreads / 32) {
-        const float* src = p.ws.partial + (static_cast<size_t>(bh) * p.gstride + a) * p.nchunk * (d + 2);
-        float M = -INFINITY;
-        for (int c = lane; c < p.nchunk; c += 32) M = fmaxf(M, __ldcg(src + static_cast<size_t>(c) * (d + 2)));
-#pragma unroll
-        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float L = 0.f;
-        for (int c = lane; c < p.nchunk; c += 32) {
-            float mc = __ldcg(src + static_cast<size_t>(c) * (d + 2));
-            if (mc != -INFINITY) L += exp2f(mc - M) * __ldcg(src + static_cast<size_t>(c) * (d + 2) + 1);
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        Tin* orow = reinterpret_cast<Tin*>(p.out) + (static_cast<size_t>(bh) * T + gq[a]) * d;
-        for (int c = lane; c < d; c += 32) {
-            float t = 0.f;
-            for (int ch = 0; ch < p.nchunk; ++ch) {
-                float mc = __ldcg(src + static_cast<size_t>(ch) * (d + 2));
-                if (mc != -INFINITY) t += exp2f(mc - M) * __ldcg(src + static_cast<size_t>(ch) * (d + 2) + 2 + c);
-            }
-            store_from_float(orow + c, t * inv);
-        }
-    }
+    merge_partials<Tin>(p, bh, nq, gq, d);
     if (tid == 0) p.ws.counters[bh] = 0;  // ready for the next call
 }
 
@@ -278,27 +295,7 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_bf16_kernel(const __gr
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int a = warp; a < nq; a += kGrThreads / 32) {
-        const float* src = p.ws.partial + (static_cast<size_t>(bh) * p.gstride + a) * p.nchunk * 66;
-        float M = -INFINITY;
-        for (int c = lane; c < p.nchunk; c += 32) M = fmaxf(M, __ldcg(src + static_cast<size_t>(c) * 66));
-#pragma unroll
-        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float L = 0.f, ax = 0.f, ay = 0.f;
-        for (int c = 0; c < p.nchunk; ++c) {
-            const float* pc = src + static_cast<size_t>(c) * 66;
-            const float mc = __ldcg(pc);
-            if (mc == -INFINITY) continue;
-            const float f = exp2f(mc - M);
-            L = fmaf(f, __ldcg(pc + 1), L);
-            ax = fmaf(f, __ldcg(pc + 2 + 2 * lane), ax);
-            ay = fmaf(f, __ldcg(pc + 3 + 2 * lane), ay);
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + base + static_cast<size_t>(gq[a]) * 64;
-        *reinterpret_cast<__nv_bfloat162*>(orow + 2 * lane) = __floats2bfloat162_rn(ax * inv, ay * inv);
-    }
+    merge_partials<__nv_bfloat16>(p, bh, nq, gq, 64);
     if (tid == 0) p.ws.counters[bh] = 0;
 }
 
