@@ -152,12 +152,10 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     uint64_t* xbar = &bars[kBarXchg + wq];
     uint32_t blk_it = 0, x_cnt = 0;
 
+    // every lane polls (each lane's own acquire), then the warp agrees on the outcome
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        __syncwarp();  // memory order for the other lanes
-        return ok != 0;
+        const bool ok = mbar_wait(bar, parity, abort_flag);
+        return __all_sync(0xffffffffu, ok);
     };
     // block j's product O += P V has completed (barrier of P buffer j % 2)
     auto wait_pv = [&](uint32_t j) -> bool { return wait_warp(&bars[kBarOFull + (j & 1u)], (j >> 1) & 1u); };
@@ -184,18 +182,27 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
             if (blk < t.nbb) {
                 const int kb = t.kb_lo + blk;
                 const int j0 = t.kbase + kBN * kb;
-                uint32_t padw = 0u;
-                if (p.pad) {
-                    const int jd = j0 + c0 + lane;
-                    bool padded = false;
-                    if (jd >= 0 && jd < t.Tc)
-                        padded = p.pad[static_cast<size_t>(t.b) * p.T + t.c + static_cast<size_t>(t.dil) * jd] != 0;
-                    padw = __ballot_sync(0xffffffffu, padded);
+                // block inside the band for every row and inside [0, Tc): no per-column test
+                // (128 kb + y - x lies in [0, 2r] for all x, y in [0, 128))
+                const bool interior = !p.pad && kb >= 1 && kBN * kb + kBN - 1 <= 2 * p.r && j0 >= 0 &&
+                                      j0 + kBN <= t.Tc;
+                if (interior) {
+                    mk = 0xffffffffu;
+                    need = true;
+                } else {
+                    uint32_t padw = 0u;
+                    if (p.pad) {
+                        const int jd = j0 + c0 + lane;
+                        bool padded = false;
+                        if (jd >= 0 && jd < t.Tc)
+                            padded = p.pad[static_cast<size_t>(t.b) * p.T + t.c + static_cast<size_t>(t.dil) * jd] != 0;
+                        padw = __ballot_sync(0xffffffffu, padded);
+                    }
+                    const int ylo = max(max(0, x - kBN * kb), -j0);
+                    const int yhi = min(min(kBN, x + 2 * p.r + 1 - kBN * kb), t.Tc - j0);
+                    mk = range_bits(ylo - c0, yhi - c0) & ~padw;
+                    need = __any_sync(0xffffffffu, max(ylo, c0) < min(yhi, c0 + 32));
                 }
-                const int ylo = max(max(0, x - kBN * kb), -j0);
-                const int yhi = min(min(kBN, x + 2 * p.r + 1 - kBN * kb), t.Tc - j0);
-                mk = range_bits(ylo - c0, yhi - c0) & ~padw;
-                need = __any_sync(0xffffffffu, max(ylo, c0) < min(yhi, c0 + 32));
             } else {
                 const int gb = blk - t.nbb;
                 ncols = global_block_cols(t.ngk, gb);
