@@ -14,35 +14,31 @@
 // U G).
 //
 // Per key block:   S = Q K^T        tcgen05.mma, M=128, N=128 (or the global
-//                                   count rounded to 16), K=64 -> TMEM (fp32),
-//                                   double-buffered so the next block's S is
-//                                   computed during this block's softmax
-//                  online softmax   four threads per query row, one per
-//                                   quarter (32 keys) of the block; each
-//                                   keeps its own running max, exponent base
-//                                   and row sum (fp32, log2 domain)
-//                  O_q += P_q V_q   P (bf16) through 128B-swizzled shared
-//                                   memory (double-buffered); k-steps 2q and
-//                                   2q+1 of the PV product (keys 32q..32q+31)
-//                                   accumulate into O_q, so each quarter's
-//                                   exponent base stays private; M=128, N=64
-// A quarter's base only moves (O_q and its sum rescaled in place) when its
-// running max exceeds the base by more than 2^8; otherwise p = 2^(s - base)
-// stays below 256, which fp32 accumulation and bf16 P absorb.  At the end of
-// a tile the quarters swap (base, sum) once and each writes 16 output
-// columns: y = sum_q 2^(m_q - M) O_q / sum_q 2^(m_q - M) l_q.
+//                                   count rounded to 16), K=64, operands in
+//                                   shared memory -> S in TMEM (fp32)
+//                  online softmax   one thread per query row (TMEM lane), all
+//                                   128 columns of the block in registers;
+//                                   running max, exponent base and row sum
+//                                   in fp32, log2 domain
+//                  O += P V         P (bf16) written back to TMEM by the
+//                                   softmax threads and read from there as
+//                                   the A operand; V from shared memory;
+//                                   M=128, N=64, K=128
+// The exponent base only moves (O and the row sum rescaled in place) when a
+// block's max exceeds it by more than 2^8; otherwise p = 2^(s - base) stays
+// below 256, which fp32 accumulation and bf16 P absorb.
 // The mask view of the note ("Mask View": A = QK^T/sqrt(d) + M, M = -inf off
 // the pattern) is applied inline: band limits and sequence ends as a per-row
 // column interval, padded keys from the key padding mask, the global-key
-// dedup test per column.  Nothing of size T x T is built.
+// dedup test per column.  Blocks that lie inside every row's window need no
+// test at all.  Nothing of size T x T is built.
 //
-// Warp roles (640 threads): warp 0 lane 0 TMA producer, warp 1 lane 0 issues
-// S = Q K^T (warp 1 also owns the TMEM allocation), warps 2 and 3 lane 0
-// issue the two halves of the PV product, warps 4..19 softmax: quarter (w - 4) / 4 of TMEM lanes 32*(w%4)..+31, so every SM
-// sub-partition runs four softmax warps.  Every hand-off is an mbarrier and
-// every wait is bounded (ptx.cuh).  In steady state no softmax warp waits on
-// a round trip through the MMA warp: S is double-buffered, and P(k) only
-// needs the product of block k-2 to have finished.
+// Two CTAs share an SM (96 KB of shared memory and 256 TMEM columns each):
+// while one CTA's softmax warps wait on a barrier or a TMEM load, the
+// other's keep the exponent unit busy.  Warp roles (192 threads): warp 0
+// lane 0 TMA producer, warp 1 TMEM owner and lane 0 MMA issuer, warps 2..5
+// softmax (TMEM lanes 32*(w%4)..+31).  Every hand-off is an mbarrier and
+// every wait is bounded (ptx.cuh).
 #pragma once
 #include "lf_common.cuh"
 #include "ptx.cuh"
@@ -52,41 +48,41 @@ namespace lf {
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kHD = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 2;                 // Q, K and V rings
 constexpr int kTileBytes = kBM * kHD * 2;  // 16 KB: 128 rows x 128 bytes
-constexpr int kBandThreads = 640;
-constexpr int kSoftmaxWarp0 = 4;           // warps 4..19
-constexpr int kSoftmaxWarps = 16;
-constexpr float kRescaleLog2 = 8.f;        // move the exponent base only past 2^8
+constexpr int kBandThreads = 192;
+constexpr int kBandCtasPerSm = 2;
+constexpr int kSoftmaxWarp0 = 2;  // warps 2..5
+constexpr int kSoftmaxWarps = 4;
+constexpr float kRescaleLog2 = 8.f;  // move the exponent base only past 2^8
 
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTileBytes;                  // kStages x 16 KB
-constexpr int kOffV = kOffK + kStages * kTileBytes;        // kStages x 16 KB
-constexpr int kOffP = kOffV + kStages * kTileBytes;        // 2 buffers x (keys 0..63 | 64..127) x 16 KB
-constexpr int kOffX = kOffP + 2 * 2 * kTileBytes;          // per-tile exchange: [2 parity][2 (m, l)][4 q][128] f32
-constexpr int kOffBar = kOffX + 2 * 2 * 4 * kBM * 4;
+constexpr int kOffK = kOffQ + kStages * kTileBytes;
+constexpr int kOffV = kOffK + kStages * kTileBytes;
+constexpr int kOffBar = kOffV + kStages * kTileBytes;
 // barrier slots
-constexpr int kBarQFull = 0, kBarQEmpty = 1, kBarKvFull = 2, kBarKvEmpty = kBarKvFull + kStages,
-              kBarSFull = kBarKvEmpty + kStages, kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2,
-              kBarOFull = kBarPFull + 2, kBarXchg = kBarOFull + 2, kBarDrain = kBarXchg + 4,
-              kNumBars = kBarDrain + 1;
+constexpr int kBarQFull = 0, kBarQEmpty = kBarQFull + kStages, kBarKFull = kBarQEmpty + kStages,
+              kBarKEmpty = kBarKFull + kStages, kBarVFull = kBarKEmpty + kStages, kBarVEmpty = kBarVFull + kStages,
+              kBarSFull = kBarVEmpty + kStages, kBarSFree = kBarSFull + 1, kBarPFull = kBarSFree + 1,
+              kBarOFull = kBarPFull + 1, kBarDrain = kBarOFull + 1, kNumBars = kBarDrain + 1;
 constexpr int kOffMisc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
 constexpr int kMiscBytes = 16;
 constexpr int kBandSmem = kOffMisc + kMiscBytes + 1024;  // + alignment slack
-static_assert(kBandSmem <= 232448, "shared memory budget");
+static_assert(kBandCtasPerSm * (kBandSmem + 1024) <= 233472, "shared memory budget for two CTAs per SM");
 
-constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S buffers at 0 and 128 (fp32, 128 wide); output accumulator
-// O_q of key quarter q at 256 + 64 q (fp32, 64 wide).
-__device__ __forceinline__ uint32_t col_s(uint32_t buf) { return buf * 128u; }
-__device__ __forceinline__ uint32_t col_o(uint32_t q) { return 256u + 64u * q; }
+// TMEM columns (256 per CTA): S (fp32, 128 wide) at 0, P (bf16 pairs, 64
+// wide) at 128, O (fp32, 64 wide) at 192.
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
 
 struct BandTile {
     int b, bh, c, dil, dk, R;
     int Tc, q0, kbase, kb_lo, nbb, ngk, ngb;
 };
 
-__device__ __forceinline__ BandTile band_decode(const BandTcParams& p, int item) {
+// Out of line: every role walks the same tiles, and one copy of this code
+// (integer divisions included) keeps the kernel small.
+__device__ __noinline__ BandTile band_decode(const BandTcParams& p, int item) {
     BandTile t;
     t.b = item / p.items_per_b;
     int rem = item - t.b * p.items_per_b;
@@ -133,32 +129,307 @@ __device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
     return upto_hi & ~upto_lo;
 }
 
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Walks the (item, block) sequence of this CTA in the order every role uses.
+struct BlockCursor {
+    int item, blk, nb;
+    BandTile t;
+    __device__ __forceinline__ void start(const BandTcParams& p) {
+        item = blockIdx.x;
+        blk = 0;
+        if (item < p.n_items) {
+            t = band_decode(p, item);
+            nb = t.nbb + t.ngb;
+        } else {
+            nb = 0;
+        }
+    }
+    __device__ __forceinline__ bool valid(const BandTcParams& p) const { return item < p.n_items; }
+    __device__ __forceinline__ void next(const BandTcParams& p) {
+        if (++blk < nb) return;
+        blk = 0;
+        item += gridDim.x;
+        if (item < p.n_items) {
+            t = band_decode(p, item);
+            nb = t.nbb + t.ngb;
+        }
+    }
+};
+
+// ------------------------------------------------------------- TMA producer
+// K runs one block ahead of V: K(g + 1) is needed as soon as the softmax has
+// read S(g), V(g) only once P(g) is written.
+__device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
+                                              volatile int* abort_flag) {
+    BlockCursor kc, vc;
+    kc.start(p);
+    vc.start(p);
+    uint32_t gk = 0, gv = 0, qt = 0;
+    auto issue_k = [&]() -> bool {
+        const BandTile& t = kc.t;
+        if (kc.blk == 0) {
+            const uint32_t qs = qt & 1u;
+            if (!mbar_wait(&bars[kBarQEmpty + qs], ((qt >> 1) & 1u) ^ 1u, abort_flag)) return false;
+            mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes);
+            uint8_t* dQ = smem + kOffQ + qs * kTileBytes;
+            for (int u = 0; u < kBM; u += t.R)
+                tma_load_3d(dQ + u * 128, &p.tm_q[t.dk], &bars[kBarQFull + qs], 0, t.c + t.dil * (t.q0 + u), t.bh);
+            ++qt;
+        }
+        const uint32_t s = gk & 1u;
+        if (!mbar_wait(&bars[kBarKEmpty + s], ((gk >> 1) & 1u) ^ 1u, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bars[kBarKFull + s], kTileBytes);
+        uint8_t* dK = smem + kOffK + s * kTileBytes;
+        if (kc.blk < t.nbb) {
+            const int j0 = t.kbase + kBN * (t.kb_lo + kc.blk);
+            for (int u = 0; u < kBN; u += t.R)
+                tma_load_3d(dK + u * 128, &p.tm_k[t.dk], &bars[kBarKFull + s], 0, t.c + t.dil * (j0 + u), t.bh);
+        } else {
+            tma_load_3d(dK, &p.tm_kg, &bars[kBarKFull + s], 0, (kc.blk - t.nbb) * kBN, t.bh);
+        }
+        ++gk;
+        return true;
+    };
+    auto issue_v = [&]() -> bool {
+        const BandTile& t = vc.t;
+        const uint32_t s = gv & 1u;
+        if (!mbar_wait(&bars[kBarVEmpty + s], ((gv >> 1) & 1u) ^ 1u, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes);
+        uint8_t* dV = smem + kOffV + s * kTileBytes;
+        if (vc.blk < t.nbb) {
+            const int j0 = t.kbase + kBN * (t.kb_lo + vc.blk);
+            for (int u = 0; u < kBN; u += t.R)
+                tma_load_3d(dV + u * 128, &p.tm_v[t.dk], &bars[kBarVFull + s], 0, t.c + t.dil * (j0 + u), t.bh);
+        } else {
+            tma_load_3d(dV, &p.tm_vg, &bars[kBarVFull + s], 0, (vc.blk - t.nbb) * kBN, t.bh);
+        }
+        ++gv;
+        return true;
+    };
+    bool first = true;
+    while (vc.valid(p)) {  // K(0); then K(g + 1), V(g) for g = 0, 1, ...
+        if (kc.valid(p)) {
+            if (!issue_k()) break;
+            kc.next(p);
+            if (first) {
+                first = false;
+                continue;
+            }
+        }
+        if (!issue_v()) break;
+        vc.next(p);
+    }
+    if (*abort_flag) {  // let issued copies land before the CTA can exit
+        for (uint32_t s = 0; s < kStages; ++s) {
+            if (gk > s) (void)mbar_wait_drain(&bars[kBarKFull + s], ((gk - 1 - s) >> 1) & 1u);
+            if (gv > s) (void)mbar_wait_drain(&bars[kBarVFull + s], ((gv - 1 - s) >> 1) & 1u);
+            if (qt > s) (void)mbar_wait_drain(&bars[kBarQFull + s], ((qt - 1 - s) >> 1) & 1u);
+        }
+    }
+}
+
+// --------------------------------------------------------------- MMA issuer
+// S(g) = Q K(g)^T as soon as K(g) has landed and the softmax has read S(g-1);
+// then O += P(g-1) V(g-1) once P(g-1) is in TMEM.  The MMA pipe accepts one
+// tcgen05.mma every ~54-64 cycles, 12 per block: well inside the exponent
+// unit's ~1000 cycles per block, so one issuing thread is enough.
+__device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
+                                         volatile int* abort_flag, uint32_t tmem_base) {
+    const uint32_t idesc_s = idesc_bf16(kBM, kBN, 0, 0);
+    const uint32_t idesc_pv = idesc_bf16(kBM, kHD, 0, 1);
+    uint64_t dQ[kStages], dK[kStages], dV[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+        dQ[s] = sdesc_k_sw128(smem_u32(smem + kOffQ + s * kTileBytes));
+        dK[s] = sdesc_k_sw128(smem_u32(smem + kOffK + s * kTileBytes));
+        dV[s] = sdesc_mn_sw128(smem_u32(smem + kOffV + s * kTileBytes));
+    }
+    const uint32_t tS = tmem_base + kColS, tP = tmem_base + kColP, tO = tmem_base + kColO;
+
+    // O += P(g) V(g) over nk keys; the first block of a tile overwrites O
+    auto issue_pv = [&](uint32_t g, int nk, bool first) -> bool {
+        const uint32_t s = g & 1u;
+        if (!mbar_wait(&bars[kBarPFull], g & 1u, abort_flag) ||
+            !mbar_wait(&bars[kBarVFull + s], (g >> 1) & 1u, abort_flag))
+            return false;
+        tc_fence_after();
+        const uint64_t dv = dV[s];
+        if (nk == kBN) {
+            if (first)
+                tc_mma_ts<false>(tO, tP + 0, dv + 0, idesc_pv);
+            else
+                tc_mma_ts<true>(tO, tP + 0, dv + 0, idesc_pv);
+#pragma unroll
+            for (int k = 1; k < 8; ++k) tc_mma_ts<true>(tO, tP + 8u * k, dv + 128u * k, idesc_pv);
+        } else {  // a partial block of global keys (never the first block of a tile)
+            for (int k = 0; k < nk / 16; ++k) tc_mma_ts<true>(tO, tP + 8u * k, dv + 128u * k, idesc_pv);
+        }
+        tc_commit(&bars[kBarOFull]);
+        tc_commit(&bars[kBarVEmpty + s]);
+        return true;
+    };
+
+    BlockCursor c;
+    c.start(p);
+    uint32_t g = 0, qt = 0;
+    int prev_nk = 0;
+    bool prev_first = false;
+    for (;;) {  // S(g), then the product of block g - 1
+        const bool have = c.valid(p);
+        if (have) {
+            const BandTile& t = c.t;
+            const uint32_t qs = (qt - (c.blk == 0 ? 0u : 1u)) & 1u;
+            if (c.blk == 0) {
+                if (!mbar_wait(&bars[kBarQFull + qs], (qt >> 1) & 1u, abort_flag)) break;
+                ++qt;
+            }
+            const uint32_t s = g & 1u;
+            if (!mbar_wait(&bars[kBarKFull + s], (g >> 1) & 1u, abort_flag) ||
+                (g > 0 && !mbar_wait(&bars[kBarSFree], (g - 1) & 1u, abort_flag)))
+                break;
+            tc_fence_after();
+            const int ncols = c.blk < t.nbb ? kBN : global_block_cols(t.ngk, c.blk - t.nbb);
+            const uint32_t ids = ncols == kBN ? idesc_s : idesc_bf16(kBM, ncols, 0, 0);
+            const uint64_t dq = dQ[qs], dk = dK[s];
+            tc_mma<false>(tS, dq + 0, dk + 0, ids);  // K-steps of 16 (32 bytes = 2 units)
+            tc_mma<true>(tS, dq + 2, dk + 2, ids);
+            tc_mma<true>(tS, dq + 4, dk + 4, ids);
+            tc_mma<true>(tS, dq + 6, dk + 6, ids);
+            tc_commit(&bars[kBarSFull]);
+            tc_commit(&bars[kBarKEmpty + s]);
+            if (c.blk == c.nb - 1) tc_commit(&bars[kBarQEmpty + qs]);
+        }
+        if (g > 0 && !issue_pv(g - 1, prev_nk, prev_first)) break;
+        if (!have) break;
+        prev_nk = c.blk < c.t.nbb ? kBN : global_block_cols(c.t.ngk, c.blk - c.t.nbb);
+        prev_first = c.blk == 0;
+        ++g;
+        c.next(p);
+    }
+    tc_commit(&bars[kBarDrain]);
+}
+
 // ------------------------------------------------------------ softmax role
-// Thread (row x, quarter q) owns key columns [32 q, 32 q + 32) of every block
-// of row x.  POS: scale > 0, so maxima are taken on raw scores and the scale
-// is folded into the exp2 argument.
-template <bool POS>
-__device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
-                                             volatile int* abort_flag, uint32_t tmem_base) {
+// Thread x owns query row x of the tile (TMEM lane x) and walks each S block
+// in four chunks of 32 columns: the TMEM load of chunk c + 1 is in flight
+// while chunk c is exponentiated and its P (16 columns of bf16 pairs) is
+// stored, so only two chunks of S are ever held in registers.
+//
+// Exponent base.  p = 2^(s*sl2 - base) with base = m_ref.  The base moves
+// between blocks, to the largest scaled score seen so far, once that exceeds
+// it by more than 2^8 (O and the row sum are rescaled then; the O rescale
+// needs the previous product to have finished, which the P store waits for
+// anyway).  Inside a block the base stays put unless a chunk's max exceeds
+// it by more than 2^64, so p < 2^64 and fp32 sums stay finite; that rare
+// jump rescales O and the P chunks already stored.
+constexpr float kBigJumpLog2 = 64.f;
+
+// Multiplies the first nchunks P chunks (16 columns of bf16 pairs each) of
+// this thread's row by alpha, in TMEM.
+__device__ __forceinline__ void rescale_p_chunks(uint32_t tP, int nchunks, float alpha) {
+    tmem_st_wait();  // this thread's own stores have landed
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+        uint32_t pr[16];
+        tmem_ld16(tP + 16u * c, pr);
+        tmem_ld_wait16(pr);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&pr[u]);
+            const float2 f = __bfloat1622float2(h);
+            pr[u] = pack_bf16x2(f.x * alpha, f.y * alpha);
+        }
+        tmem_st16(tP + 16u * c, pr);
+    }
+}
+
+// Multiplies this thread's row of O (64 fp32 columns) by alpha, in TMEM.
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll 1
+    for (int part = 0; part < 4; ++part) {
+        uint32_t orr[16];
+        tmem_ld16(tO + 16u * part, orr);
+        tmem_ld_wait16(orr);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+        tmem_st16(tO + 16u * part, orr);
+    }
+}
+
+// Multiplies 16 packed bf16 pairs by alpha.
+__device__ __forceinline__ void scale_packed(uint32_t* pk, float alpha) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pk[u]));
+        pk[u] = pack_bf16x2(f.x * alpha, f.y * alpha);
+    }
+}
+
+__device__ __forceinline__ uint32_t pick4(const uint32_t* v, int c) {
+    return c == 0 ? v[0] : (c == 1 ? v[1] : (c == 2 ? v[2] : v[3]));
+}
+
+__device__ __forceinline__ void softmax_role(const BandTcParams& p, uint64_t* bars, volatile int* abort_flag,
+                                             uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wq = warp & 3;
-    const int qi = (warp - kSoftmaxWarp0) >> 2;  // key quarter
-    const int x = wq * 32 + lane;                // query row inside the tile = TMEM lane
+    const int x = wq * 32 + lane;  // query row inside the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tOq = tmem_base + lane_off + col_o(qi);
-    const int rowoff = (x >> 3) * 1024 + (x & 7) * 128;
-    const float sl2 = p.sl2;
-    float* xm = reinterpret_cast<float*>(smem + kOffX);  // [2 parity][2][4][128]
-    uint64_t* xbar = &bars[kBarXchg + wq];
-    uint32_t blk_it = 0, x_cnt = 0;
+    const uint32_t tS = tmem_base + lane_off + kColS;
+    const uint32_t tP = tmem_base + lane_off + kColP;
+    const uint32_t tO = tmem_base + lane_off + kColO;
+    // scale >= 0: maxima on raw scores (masked columns -inf); scale < 0: minima
+    // (masked columns +inf); either way the scale is folded into the exp2 FMA
+    const bool pos = p.sl2 >= 0.f;
+    const float kmul = p.sl2 == 0.f ? 1e-30f : p.sl2;
+    const uint32_t fill = __float_as_uint(pos ? -INFINITY : INFINITY);
+    uint32_t g = 0;
 
     // every lane polls (each lane's own acquire), then the warp agrees on the outcome
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
         const bool ok = mbar_wait(bar, parity, abort_flag);
         return __all_sync(0xffffffffu, ok);
     };
-    // block j's product O += P V has completed (barrier of P buffer j % 2)
-    auto wait_pv = [&](uint32_t j) -> bool { return wait_warp(&bars[kBarOFull + (j & 1u)], (j >> 1) & 1u); };
+
+    // The output row of a finished tile is written once the product that
+    // completes its O is done, which the first P store of the next tile (or
+    // the end of the role) waits for anyway.
+    bool pend = false, pend_ok = false;
+    float pend_inv = 0.f;
+    uint4* pend_dst = nullptr;
+    auto flush = [&]() {
+        if (!pend) return;
+        pend = false;
+#pragma unroll 1
+        for (int part = 0; part < 4; ++part) {
+            uint32_t o[16];
+            tmem_ld16(tO + 16u * part, o);
+            tmem_ld_wait16(o);
+            if (pend_ok) {
+                uint4 v0, v1;
+                v0.x = pack_bf16x2(__uint_as_float(o[0]) * pend_inv, __uint_as_float(o[1]) * pend_inv);
+                v0.y = pack_bf16x2(__uint_as_float(o[2]) * pend_inv, __uint_as_float(o[3]) * pend_inv);
+                v0.z = pack_bf16x2(__uint_as_float(o[4]) * pend_inv, __uint_as_float(o[5]) * pend_inv);
+                v0.w = pack_bf16x2(__uint_as_float(o[6]) * pend_inv, __uint_as_float(o[7]) * pend_inv);
+                v1.x = pack_bf16x2(__uint_as_float(o[8]) * pend_inv, __uint_as_float(o[9]) * pend_inv);
+                v1.y = pack_bf16x2(__uint_as_float(o[10]) * pend_inv, __uint_as_float(o[11]) * pend_inv);
+                v1.z = pack_bf16x2(__uint_as_float(o[12]) * pend_inv, __uint_as_float(o[13]) * pend_inv);
+                v1.w = pack_bf16x2(__uint_as_float(o[14]) * pend_inv, __uint_as_float(o[15]) * pend_inv);
+                pend_dst[2 * part] = v0;
+                pend_dst[2 * part + 1] = v1;
+            }
+        }
+    };
 
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
         const BandTile t = band_decode(p, item);
@@ -168,319 +439,194 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
         if (row_ok && ((p.gbit[static_cast<size_t>(t.b) * p.W + (i >> 5)] >> (i & 31)) & 1u)) row_ok = false;
         const int32_t* gk = p.gk_list + static_cast<size_t>(t.b) * p.gstride;
         const int reach = t.dil * p.r;
+        // the first block of global keys, one key per lane and chunk, fetched early
+        uint32_t kreg[4] = {0u, 0u, 0u, 0u};
+        if (t.ngb > 0) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                if (32 * w + lane < t.ngk) kreg[w] = static_cast<uint32_t>(__ldg(gk + 32 * w + lane));
+        }
 
-        float m_run = -INFINITY;  // running max of this quarter (scaled, log2 domain)
-        float m_ref = -INFINITY;  // its exponent base (-inf: nothing valid yet)
-        float l_q = 0.f;          // its row sum, relative to m_ref
+        float m_ref = -INFINITY;   // exponent base (scaled, log2 domain; -inf: nothing valid yet)
+        float m_seen = -INFINITY;  // largest scaled score seen so far
+        float l_row = 0.f;         // row sum relative to m_ref
         const int nb = t.nbb + t.ngb;
-        for (int blk = 0; blk < nb; ++blk, ++blk_it) {
-            const uint32_t sb = blk_it & 1u;
-            const int c0 = 32 * qi;
-            uint32_t mk = 0u;
-            bool need;
-            int ncols = kBN;
-            if (blk < t.nbb) {
-                const int kb = t.kb_lo + blk;
-                const int j0 = t.kbase + kBN * kb;
-                // block inside the band for every row and inside [0, Tc): no per-column test
-                // (128 kb + y - x lies in [0, 2r] for all x, y in [0, 128))
-                const bool interior = !p.pad && kb >= 1 && kBN * kb + kBN - 1 <= 2 * p.r && j0 >= 0 &&
-                                      j0 + kBN <= t.Tc;
-                if (interior) {
-                    mk = 0xffffffffu;
-                    need = true;
-                } else {
-                    uint32_t padw = 0u;
-                    if (p.pad) {
-                        const int jd = j0 + c0 + lane;
-                        bool padded = false;
+        for (int blk = 0; blk < nb; ++blk, ++g) {
+            // ---- which columns this row keeps: band blocks inside every row's window and
+            //      inside [0, Tc) need no test (128 kb + y - x lies in [0, 2r] for all x, y)
+            const bool band = blk < t.nbb;
+            const int kb = t.kb_lo + blk;
+            const int j0 = t.kbase + kBN * kb;
+            const bool interior =
+                band && !p.pad && kb >= 1 && kBN * kb + kBN - 1 <= 2 * p.r && j0 >= 0 && j0 + kBN <= t.Tc;
+            const int ylo = max(max(0, x - kBN * kb), -j0);  // band: kept columns [ylo, yhi)
+            const int yhi = min(min(kBN, x + 2 * p.r + 1 - kBN * kb), t.Tc - j0);
+            uint32_t padv[4] = {0u, 0u, 0u, 0u};  // band: key padding of column 32 w + lane
+            int nch = 4, nvalid = kBN;
+            if (band) {
+                if (p.pad) {
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int jd = j0 + 32 * w + lane;
                         if (jd >= 0 && jd < t.Tc)
-                            padded = p.pad[static_cast<size_t>(t.b) * p.T + t.c + static_cast<size_t>(t.dil) * jd] != 0;
-                        padw = __ballot_sync(0xffffffffu, padded);
+                            padv[w] = p.pad[static_cast<size_t>(t.b) * p.T + t.c + static_cast<size_t>(t.dil) * jd];
                     }
-                    const int ylo = max(max(0, x - kBN * kb), -j0);
-                    const int yhi = min(min(kBN, x + 2 * p.r + 1 - kBN * kb), t.Tc - j0);
-                    mk = range_bits(ylo - c0, yhi - c0) & ~padw;
-                    need = __any_sync(0xffffffffu, max(ylo, c0) < min(yhi, c0 + 32));
                 }
             } else {
                 const int gb = blk - t.nbb;
-                ncols = global_block_cols(t.ngk, gb);
-                const int nvalid = min(kBN, t.ngk - gb * kBN);
-                need = c0 < nvalid;
-                if (need) {
-                    for (int a = 0; a < 32 && c0 + a < nvalid; ++a) {
-                        const int diff = __ldg(gk + gb * kBN + c0 + a) - i;
-                        const bool in_window = (diff % t.dil == 0) && diff <= reach && diff >= -reach;
-                        if (!in_window) mk |= 1u << a;
-                    }
+                nvalid = min(kBN, t.ngk - gb * kBN);
+                nch = (nvalid + 31) >> 5;
+                if (gb > 0) {
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        kreg[w] = 32 * w + lane < nvalid ? static_cast<uint32_t>(__ldg(gk + gb * kBN + 32 * w + lane)) : 0u;
                 }
             }
-            const bool full = __all_sync(0xffffffffu, mk == 0xffffffffu);
 
-            // ---- this quarter of the S block
-            if (!wait_warp(&bars[kBarSFull + sb], (blk_it >> 1) & 1u)) return;
+            // ---- deferred base move (decided on the blocks before this one)
+            float alpha_o = 1.f;
+            const bool o_move = m_ref != -INFINITY && m_seen > m_ref + kRescaleLog2;
+            if (o_move) {
+                alpha_o = ex2_approx(m_ref - m_seen);
+                m_ref = m_seen;
+                l_row *= alpha_o;
+            }
+            const bool warp_o_move = __any_sync(0xffffffffu, o_move);
+            // P may be overwritten (and O touched) once the previous product is done
+            bool p_ready = false;
+            auto ensure_p_ready = [&]() -> bool {
+                if (p_ready) return true;
+                if (g > 0) {
+                    if (!wait_warp(&bars[kBarOFull], (g - 1) & 1u)) return false;
+                    tc_fence_after();
+                }
+                flush();
+                if (warp_o_move) rescale_o(tO, alpha_o);
+                p_ready = true;
+                return true;
+            };
+
+            if (!wait_warp(&bars[kBarSFull], g & 1u)) return;
             tc_fence_after();
-            uint32_t sr[32];
-            if (need) tmem_ld32(tmem_base + lane_off + col_s(sb) + 32u * qi, sr);
-            tmem_ld_wait(sr);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kBarSFree + sb]);
-
-            float mx = -INFINITY;
-            if (need) {
-                float mxp[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) mxp[u] = -INFINITY;
-                if (full) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        float f = __uint_as_float(sr[j]);
-                        if (!POS) f *= sl2;
-                        sr[j] = __float_as_uint(f);
-                        mxp[j & 7] = fmaxf(mxp[j & 7], f);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        float f = __uint_as_float(sr[j]);
-                        if (!POS) f *= sl2;
-                        f = ((mk >> j) & 1u) ? f : -INFINITY;
-                        sr[j] = __float_as_uint(f);
-                        mxp[j & 7] = fmaxf(mxp[j & 7], f);
-                    }
-                }
-                mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                           fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
-                if (POS) mx *= sl2;  // -inf stays -inf
-            }
-            m_run = fmaxf(m_run, mx);
-
-            // ---- move this quarter's exponent base if its max ran past it (rare)
-            float alpha = 1.f;
-            bool move = (m_run != -INFINITY) && (m_ref == -INFINITY || m_run > m_ref + kRescaleLog2);
-            if (blk == 0) {
-                m_ref = m_run;  // the first product of the tile overwrites O_q
-                move = false;
-            } else if (move) {
-                alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_run);
-                m_ref = m_run;
-                l_q *= alpha;
-            }
-            if (__any_sync(0xffffffffu, move)) {
-                if (!wait_pv(blk_it - 1)) return;  // O_q holds every earlier product
-                tc_fence_after();
-                uint32_t orr[32];
-#pragma unroll 1
-                for (int part = 0; part < 2; ++part) {
-                    tmem_ld32(tOq + 32u * part, orr);
-                    tmem_ld_wait(orr);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-                    tmem_st32(tOq + 32u * part, orr);
-                }
-                tmem_st_wait();
-            }
-            const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
-
-            // ---- p = 2^(s - base) as bf16 into P buffer sb (free once block blk_it - 2's product is done)
-            uint32_t pk[16];
+            uint32_t sa[32], sb[32], pka[16], pkb[16];
+            tmem_ld32(tS, sa);
             float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-            if (need) {
+            // chunk c of the block: scores in cur (the next chunk loads into nxt), P into pk;
+            // P of chunk c - 1 (in pk_prev) is stored one chunk late
+            auto chunk = [&](uint32_t* cur, uint32_t* nxt, uint32_t* pk, uint32_t* pk_prev, const int c) -> bool {
+                tmem_ld_wait(cur);
+                if (c + 1 < nch) {
+                    tmem_ld32(tS + 32u * (c + 1), nxt);
+                } else {  // the whole S block is in registers or consumed: the MMA may overwrite it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[kBarSFree]);
+                }
+                if (!interior) {
+                    uint32_t m;
+                    if (band) {
+                        m = range_bits(ylo - 32 * c, yhi - 32 * c);
+                        if (p.pad) m &= ~__ballot_sync(0xffffffffu, pick4(padv, c) != 0u);
+                    } else {  // global keys not already in the row's window
+                        m = 0u;
+                        const uint32_t kc = pick4(kreg, c);
+                        const int na = min(32, nvalid - 32 * c);
+#pragma unroll 1
+                        for (int a = 0; a < na; ++a) {
+                            const int diff = static_cast<int>(__shfl_sync(0xffffffffu, kc, a)) - i;
+                            const bool in_window =
+                                diff <= reach && diff >= -reach && (t.dil == 1 || diff % t.dil == 0);
+                            m |= in_window ? 0u : (1u << a);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (!((m >> j) & 1u)) cur[j] = fill;
+                }
+                float mx;
+                if (pos) {
+                    float mxp[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) mxp[u] = fmaxf(__uint_as_float(cur[2 * u]), __uint_as_float(cur[2 * u + 1]));
+#pragma unroll
+                    for (int j = 8; j < 32; j += 8)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            mxp[u] = fmax3(mxp[u], __uint_as_float(cur[j + 2 * u]), __uint_as_float(cur[j + 2 * u + 1]));
+                    mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
+                } else {
+                    float mnp[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) mnp[u] = fminf(__uint_as_float(cur[2 * u]), __uint_as_float(cur[2 * u + 1]));
+#pragma unroll
+                    for (int j = 8; j < 32; j += 8)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            mnp[u] = fmin3(mnp[u], __uint_as_float(cur[j + 2 * u]), __uint_as_float(cur[j + 2 * u + 1]));
+                    mx = fminf(fminf(mnp[0], mnp[1]), fminf(mnp[2], mnp[3]));
+                }
+                mx *= kmul;  // the largest scaled score of the chunk (-inf if none is kept)
+                m_seen = fmaxf(m_seen, mx);
+                if (m_ref == -INFINITY) m_ref = mx;  // everything so far had zero weight
+                const bool big = mx > m_ref + kBigJumpLog2;
+                if (__any_sync(0xffffffffu, big)) {  // rare: rescale what this block already holds
+                    const float alpha = big ? ex2_approx(m_ref - mx) : 1.f;
+                    if (big) {
+                        m_ref = mx;
+                        l_row *= alpha;
+                        lsum[0] *= alpha;
+                        lsum[1] *= alpha;
+                        lsum[2] *= alpha;
+                        lsum[3] *= alpha;
+                    }
+                    if (c > 0) scale_packed(pk_prev, alpha);
+                    if (c > 1) rescale_p_chunks(tP, c - 1, alpha);
+                    if (blk > 0) {
+                        if (!ensure_p_ready()) return false;
+                        rescale_o(tO, alpha);
+                    }
+                }
+                const float nb2 = (m_ref == -INFINITY) ? 0.f : -m_ref;
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
-                    const float v0 = __uint_as_float(sr[j]), v1 = __uint_as_float(sr[j + 1]);
-                    const float e0 = POS ? ex2_approx(fmaf(v0, sl2, -base)) : ex2_approx(v0 - base);
-                    const float e1 = POS ? ex2_approx(fmaf(v1, sl2, -base)) : ex2_approx(v1 - base);
+                    const float e0 = ex2_approx(fmaf(__uint_as_float(cur[j]), kmul, nb2));
+                    const float e1 = ex2_approx(fmaf(__uint_as_float(cur[j + 1]), kmul, nb2));
                     lsum[(j >> 1) & 3] += e0 + e1;
                     pk[j >> 1] = pack_bf16x2(e0, e1);
                 }
-            } else {
-#pragma unroll
-                for (int u = 0; u < 16; ++u) pk[u] = 0u;
-            }
-            l_q += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
-            if (blk_it >= 2 && !wait_pv(blk_it - 2)) return;
-            uint8_t* psub = smem + kOffP + sb * (2 * kTileBytes) + (qi >> 1) * kTileBytes + rowoff;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (c0 + 8 * u < ncols) {
-                    const int ch = ((qi & 1) << 2) + u;  // 16-byte chunk inside the 128-byte row
-                    *reinterpret_cast<uint4*>(psub + ((ch ^ (x & 7)) << 4)) =
-                        make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                if (c > 0) {
+                    if (!ensure_p_ready()) return false;
+                    tmem_st16(tP + 16u * (c - 1), pk_prev);
                 }
+                return true;
+            };
+#pragma unroll 1
+            for (int c = 0; c < nch; c += 2) {
+                if (!chunk(sa, sb, pka, pkb, c)) return;
+                if (c + 1 < nch && !chunk(sb, sa, pkb, pka, c + 1)) return;
             }
-            fence_proxy_async_smem();
+            if (!ensure_p_ready()) return;
+            tmem_st16(tP + 16u * (nch - 1), (nch & 1) ? pka : pkb);
+            l_row += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kBarPFull + sb]);
+            if (lane == 0) mbar_arrive(&bars[kBarPFull]);
         }
-
-        // ---- epilogue: the four quarters swap (base, sum); this thread writes output
-        //      columns [16 q, 16 q + 16) of its row (global rows are written by K2)
-        float* slot = xm + (x_cnt & 1u) * (2 * 4 * kBM);
-        slot[qi * kBM + x] = m_ref;
-        slot[4 * kBM + qi * kBM + x] = l_q;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(xbar);
-        if (!wait_warp(xbar, x_cnt & 1u)) return;
-        ++x_cnt;
-        float mq[4], lq[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            mq[u] = slot[u * kBM + x];
-            lq[u] = slot[4 * kBM + u * kBM + x];
-        }
-        const float M = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-        float wgt[4], L = 0.f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            wgt[u] = (mq[u] == -INFINITY) ? 0.f : ex2_approx(mq[u] - M);
-            L = fmaf(wgt[u], lq[u], L);
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        if (!wait_pv(blk_it - 1)) return;
+        // ---- this tile's rows: y = O / l, written once its last product is done
+        pend = true;
+        pend_ok = row_ok;
+        pend_inv = l_row > 0.f ? 1.f / l_row : 0.f;
+        pend_dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t.bh) * p.T + i) * kHD);
+    }
+    if (g > 0) {
+        if (!wait_warp(&bars[kBarOFull], (g - 1) & 1u)) return;
         tc_fence_after();
-        float y[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) y[c] = 0.f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            uint32_t a[16];
-            tmem_ld16(tmem_base + lane_off + col_o(u) + 16u * qi, a);
-            tmem_ld_wait16(a);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) y[c] = fmaf(wgt[u], __uint_as_float(a[c]), y[c]);
-        }
-        tc_fence_before();
-        if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t.bh) * p.T + i) * kHD + 16 * qi);
-#pragma unroll
-            for (int v8 = 0; v8 < 2; ++v8) {
-                uint4 val;
-                val.x = pack_bf16x2(y[8 * v8 + 0] * inv, y[8 * v8 + 1] * inv);
-                val.y = pack_bf16x2(y[8 * v8 + 2] * inv, y[8 * v8 + 3] * inv);
-                val.z = pack_bf16x2(y[8 * v8 + 4] * inv, y[8 * v8 + 5] * inv);
-                val.w = pack_bf16x2(y[8 * v8 + 6] * inv, y[8 * v8 + 7] * inv);
-                dst[v8] = val;
-            }
-        }
+        flush();
     }
 }
 
-// --------------------------------------------------------------- MMA roles
-// The MMA pipe accepts one tcgen05.mma every ~54 cycles at best, and an
-// issuing thread shares its SM sub-partition with four softmax warps, so the
-// work is split over three threads on three sub-partitions (S, and the two
-// halves of the PV product), and the issue path is kept free of arithmetic:
-// shared-memory descriptors are built once per stage / buffer and advanced
-// by constants (the start-address field counts 16-byte units), k-loops are
-// unrolled and the accumulate flags are literals.
-constexpr uint64_t kTile16 = kTileBytes >> 4;  // one 16 KB tile in descriptor units
-
-// S = Q K^T for every key block, in order.  The stage's K half is released
-// by this thread's commit (one of three arrivals on the stage's empty
-// barrier); V is released by the two product issuers.
-__device__ __forceinline__ void mma_s_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
-                                           volatile int* abort_flag, uint32_t tmem_base) {
-    const uint32_t idesc_s = idesc_bf16(kBM, kBN, 0, 0);
-    const uint64_t dQ = sdesc_k_sw128(smem_u32(smem + kOffQ));
-    uint64_t dK[kStages];
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) dK[s] = sdesc_k_sw128(smem_u32(smem + kOffK + s * kTileBytes));
-    uint32_t kv_it = 0, q_it = 0, blk_it = 0;
-    bool alive = true;
-    for (int item = blockIdx.x; item < p.n_items && alive; item += gridDim.x) {
-        const BandTile t = band_decode(p, item);
-        if (!mbar_wait(&bars[kBarQFull], q_it & 1u, abort_flag)) break;
-        ++q_it;
-        tc_fence_after();
-        const int nb = t.nbb + t.ngb;
-        for (int blk = 0; blk < nb; ++blk, ++blk_it, ++kv_it) {
-            const uint32_t s = kv_it % kStages, ph = (kv_it / kStages) & 1u;
-            const uint32_t sb = blk_it & 1u;
-            if (!mbar_wait(&bars[kBarKvFull + s], ph, abort_flag) ||
-                !mbar_wait(&bars[kBarSFree + sb], ((blk_it >> 1) & 1u) ^ 1u, abort_flag)) {
-                alive = false;
-                break;
-            }
-            tc_fence_after();
-            const int ncols = blk < t.nbb ? kBN : global_block_cols(t.ngk, blk - t.nbb);
-            const uint32_t ids = ncols == kBN ? idesc_s : idesc_bf16(kBM, ncols, 0, 0);
-            uint64_t dKs = dK[0];
-#pragma unroll
-            for (int u = 1; u < kStages; ++u)
-                if (s == static_cast<uint32_t>(u)) dKs = dK[u];
-            const uint32_t dS = tmem_base + col_s(sb);
-            tc_mma<false>(dS, dQ + 0, dKs + 0, ids);  // K-steps of 16 (32 bytes = 2 units)
-            tc_mma<true>(dS, dQ + 2, dKs + 2, ids);
-            tc_mma<true>(dS, dQ + 4, dKs + 4, ids);
-            tc_mma<true>(dS, dQ + 6, dKs + 6, ids);
-            tc_commit(&bars[kBarSFull + sb]);
-            tc_commit(&bars[kBarKvEmpty + s]);
-            if (blk == nb - 1) tc_commit(&bars[kBarQEmpty]);
-        }
-    }
-    tc_commit(&bars[kBarDrain]);
-}
-
-// O_q += P V for every key block, k-steps 4*half .. 4*half+3 (accumulators
-// O_{2 half}, O_{2 half + 1}).  Two of these threads run, one per half.
-__device__ __forceinline__ void mma_pv_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
-                                            volatile int* abort_flag, uint32_t tmem_base, int half) {
-    const uint32_t idesc_pv = idesc_bf16(kBM, kHD, 0, 1);
-    uint64_t dV[kStages];
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) dV[s] = sdesc_mn_sw128(smem_u32(smem + kOffV + s * kTileBytes));
-    // P sub-tile `half` holds keys 64 half .. 64 half + 63
-    const uint64_t dP0 = sdesc_k_sw128(smem_u32(smem + kOffP)) + half * kTile16;
-    const uint32_t t_o = tmem_base + col_o(2 * half);
-    const int ks0 = 4 * half;
-    uint32_t kv_it = 0, blk_it = 0;
-    bool alive = true;
-    for (int item = blockIdx.x; item < p.n_items && alive; item += gridDim.x) {
-        const BandTile t = band_decode(p, item);
-        const int nb = t.nbb + t.ngb;
-        for (int blk = 0; blk < nb; ++blk, ++blk_it, ++kv_it) {
-            const uint32_t s = kv_it % kStages;
-            const uint32_t pb = blk_it & 1u;
-            if (!mbar_wait(&bars[kBarPFull + pb], (blk_it >> 1) & 1u, abort_flag)) {
-                alive = false;
-                break;
-            }
-            tc_fence_after();
-            const int nk = blk < t.nbb ? kBN : global_block_cols(t.ngk, blk - t.nbb);
-            const uint64_t dP = dP0 + pb * (2 * kTile16);
-            uint64_t dVs = dV[0];
-#pragma unroll
-            for (int u = 1; u < kStages; ++u)
-                if (s == static_cast<uint32_t>(u)) dVs = dV[u];
-            dVs += ks0 * 128;  // 16 keys x 128 bytes per k-step
-            if (nk == kBN) {
-                if (blk == 0) {  // the first product of a tile overwrites the accumulators
-                    tc_mma<false>(t_o, dP + 0, dVs + 0, idesc_pv);
-                    tc_mma<true>(t_o, dP + 2, dVs + 128, idesc_pv);
-                    tc_mma<false>(t_o + 64u, dP + 4, dVs + 256, idesc_pv);
-                    tc_mma<true>(t_o + 64u, dP + 6, dVs + 384, idesc_pv);
-                } else {
-                    tc_mma<true>(t_o, dP + 0, dVs + 0, idesc_pv);
-                    tc_mma<true>(t_o, dP + 2, dVs + 128, idesc_pv);
-                    tc_mma<true>(t_o + 64u, dP + 4, dVs + 256, idesc_pv);
-                    tc_mma<true>(t_o + 64u, dP + 6, dVs + 384, idesc_pv);
-                }
-            } else {  // a partial block of global keys (never the first block of a tile)
-                for (int k = 0; k < 4 && ks0 + k < nk / 16; ++k)
-                    tc_mma<true>(t_o + 64u * (k >> 1), dP + 2 * k, dVs + 128 * k, idesc_pv);
-            }
-            tc_commit(&bars[kBarOFull + pb]);
-            tc_commit(&bars[kBarKvEmpty + s]);
-        }
-    }
-    tc_commit(&bars[kBarDrain]);
-}
-
-__global__ void __launch_bounds__(kBandThreads, 1) band_tc_kernel(const __grid_constant__ BandTcParams p) {
+__global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(const __grid_constant__ BandTcParams p) {
     extern __shared__ uint8_t band_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(band_smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -492,20 +638,19 @@ __global__ void __launch_bounds__(kBandThreads, 1) band_tc_kernel(const __grid_c
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[kBarQFull], 1);
-        mbar_init(&bars[kBarQEmpty], 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&bars[kBarKvFull + s], 1);
-            mbar_init(&bars[kBarKvEmpty + s], 3);  // S issuer + two PV issuers
+            mbar_init(&bars[kBarQFull + s], 1);
+            mbar_init(&bars[kBarQEmpty + s], 1);
+            mbar_init(&bars[kBarKFull + s], 1);
+            mbar_init(&bars[kBarKEmpty + s], 1);
+            mbar_init(&bars[kBarVFull + s], 1);
+            mbar_init(&bars[kBarVEmpty + s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars[kBarSFull + s], 1);
-            mbar_init(&bars[kBarSFree + s], kSoftmaxWarps);
-            mbar_init(&bars[kBarPFull + s], kSoftmaxWarps);
-            mbar_init(&bars[kBarOFull + s], 2);  // two PV issuers
-        }
-        for (int w = 0; w < 4; ++w) mbar_init(&bars[kBarXchg + w], 4);
-        mbar_init(&bars[kBarDrain], 3);
+        mbar_init(&bars[kBarSFull], 1);
+        mbar_init(&bars[kBarSFree], kSoftmaxWarps);
+        mbar_init(&bars[kBarPFull], kSoftmaxWarps);
+        mbar_init(&bars[kBarOFull], 1);
+        mbar_init(&bars[kBarDrain], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -528,63 +673,16 @@ __global__ void __launch_bounds__(kBandThreads, 1) band_tc_kernel(const __grid_c
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            uint32_t kv_it = 0, q_it = 0;
-            bool alive = true;
-            for (int item = blockIdx.x; item < p.n_items && alive; item += gridDim.x) {
-                const BandTile t = band_decode(p, item);
-                if (!mbar_wait(&bars[kBarQEmpty], (q_it & 1u) ^ 1u, abort_flag)) break;
-                ++q_it;
-                mbar_arrive_expect_tx(&bars[kBarQFull], kTileBytes);
-                for (int u = 0; u < kBM; u += t.R)
-                    tma_load_3d(smem + kOffQ + u * 128, &p.tm_q[t.dk], &bars[kBarQFull], 0,
-                                t.c + t.dil * (t.q0 + u), t.bh);
-                const int nb = t.nbb + t.ngb;
-                for (int blk = 0; blk < nb; ++blk) {
-                    const uint32_t s = kv_it % kStages, ph = (kv_it / kStages) & 1u;
-                    if (!mbar_wait(&bars[kBarKvEmpty + s], ph ^ 1u, abort_flag)) {
-                        alive = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * kTileBytes);
-                    uint8_t* dK = smem + kOffK + s * kTileBytes;
-                    uint8_t* dV = smem + kOffV + s * kTileBytes;
-                    if (blk < t.nbb) {
-                        const int j0 = t.kbase + kBN * (t.kb_lo + blk);
-                        for (int u = 0; u < kBN; u += t.R) {
-                            const int y = t.c + t.dil * (j0 + u);
-                            tma_load_3d(dK + u * 128, &p.tm_k[t.dk], &bars[kBarKvFull + s], 0, y, t.bh);
-                            tma_load_3d(dV + u * 128, &p.tm_v[t.dk], &bars[kBarKvFull + s], 0, y, t.bh);
-                        }
-                    } else {
-                        const int gb = blk - t.nbb;
-                        tma_load_3d(dK, &p.tm_kg, &bars[kBarKvFull + s], 0, gb * kBN, t.bh);
-                        tma_load_3d(dV, &p.tm_vg, &bars[kBarKvFull + s], 0, gb * kBN, t.bh);
-                    }
-                    ++kv_it;
-                }
-            }
-            if (*abort_flag) {  // let issued copies land before the CTA can exit
-                for (uint32_t s = 0; s < kStages && kv_it > s; ++s)
-                    (void)mbar_wait_drain(&bars[kBarKvFull + s], ((kv_it - 1 - s) / kStages) & 1u);
-                if (q_it) (void)mbar_wait_drain(&bars[kBarQFull], (q_it - 1) & 1u);
-            }
-        }
+        if (lane == 0) producer_role(p, smem, bars, abort_flag);
     } else if (warp == 1) {
-        if (lane == 0) mma_s_role(p, smem, bars, abort_flag, tmem_base);
-    } else if (warp < kSoftmaxWarp0) {
-        if (lane == 0) mma_pv_role(p, smem, bars, abort_flag, tmem_base, warp - 2);
+        if (lane == 0) mma_role(p, smem, bars, abort_flag, tmem_base);
     } else {
-        if (p.sl2 > 0.f)
-            softmax_role<true>(p, smem, bars, abort_flag, tmem_base);
-        else
-            softmax_role<false>(p, smem, bars, abort_flag, tmem_base);
+        softmax_role(p, bars, abort_flag, tmem_base);
     }
 
     tc_fence_before();
     __syncthreads();
-    // every MMA of the three issuers has completed before TMEM is released
+    // every MMA has completed before TMEM is released
     if (threadIdx.x == 32) (void)mbar_wait_drain(&bars[kBarDrain], 0u);
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, kStatusTimeout);

@@ -82,6 +82,27 @@ bool is_capturing(cudaStream_t s) {
     return st != cudaStreamCaptureStatusNone;
 }
 
+// Shared-memory limits of every kernel, and the carveout that lets two band
+// CTAs share an SM.
+lf_status set_kernel_attributes() {
+    const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + kMaxGlobal) * 4;
+    const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
+    if (cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) != cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrBf16Smem) !=
+            cudaSuccess)
+        return LF_ERR_CUDA;
+    return LF_OK;
+}
+
 lf_status device_state(DeviceState** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_CUDA;
@@ -93,23 +114,7 @@ lf_status device_state(DeviceState** out) {
         s.sm_count = prop.multiProcessorCount;
         if (cudaMalloc(&s.status, 256) != cudaSuccess) return LF_ERR_NO_MEMORY;
         if (cudaMemset(s.status, 0, 256) != cudaSuccess) return LF_ERR_CUDA;
-        if (cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) !=
-            cudaSuccess)
-            return LF_ERR_CUDA;
-        const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + kMaxGlobal) * 4;
-        if (cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) !=
-            cudaSuccess)
-            return LF_ERR_CUDA;
-        const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
-        if (cudaFuncSetAttribute(global_rows_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gr_max) != cudaSuccess ||
-            cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gr_max) != cudaSuccess ||
-            cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gr_max) != cudaSuccess ||
-            cudaFuncSetAttribute(global_rows_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGrBf16Smem) != cudaSuccess)
-            return LF_ERR_CUDA;
+        if (set_kernel_attributes() != LF_OK) return LF_ERR_CUDA;
         s.init = true;
     }
     *out = &s;
@@ -323,7 +328,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         bp.sl2 = sl2;
         bp.items_per_b = items_per_b;
         bp.n_items = items_per_b * B;
-        const int grid = std::min(bp.n_items, ds->sm_count);
+        const int grid = std::min(bp.n_items, kBandCtasPerSm * ds->sm_count);
         band_tc_kernel<<<grid, kBandThreads, kBandSmem, stream>>>(bp);
         ++launches;
     }
@@ -387,20 +392,7 @@ lf_status static_state(StaticState** out) {
         if (prop.major < 10) return LF_ERR_UNSUPPORTED;
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return LF_ERR_CUDA;
-        const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + kMaxGlobal) * 4;
-        const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
-        if (cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) != cudaSuccess ||
-            cudaFuncSetAttribute(global_rows_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gr_max) != cudaSuccess ||
-            cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gr_max) != cudaSuccess ||
-            cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gr_max) != cudaSuccess ||
-            cudaFuncSetAttribute(global_rows_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGrBf16Smem) != cudaSuccess)
-            return LF_ERR_CUDA;
+        if (set_kernel_attributes() != LF_OK) return LF_ERR_CUDA;
         s.sm_count = prop.multiProcessorCount;
         s.scratch = static_cast<uint8_t*>(ptr);
         s.init = true;

@@ -55,9 +55,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete.  Returns
 // false (and raises *abort) after LF_WAIT_NS, or if another role already
-// raised *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+// raised *abort.  The polling loop is out of line: only the first test is
+// inlined at each call site, which keeps the kernels' code small.
+__device__ __noinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, volatile int* abort) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -69,6 +69,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
             }
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_poll(bar, parity, abort);
 }
 
 // Bounded wait that ignores the abort flag: used on the way out, for copies
@@ -148,6 +152,18 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
     else
         asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 0;" ::"r"(d_tmem), "l"(adesc), "l"(bdesc),
                      "r"(idesc));
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]: A (M rows = TMEM lanes, K elements
+// packed two bf16 per 32-bit column, lower half first) read from TMEM.
+template <bool ACC>
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc) {
+    if (ACC)
+        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 1;" ::"r"(d_tmem), "r"(a_tmem),
+                     "l"(bdesc), "r"(idesc));
+    else
+        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 0;" ::"r"(d_tmem), "r"(a_tmem),
+                     "l"(bdesc), "r"(idesc));
 }
 
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.

@@ -116,6 +116,20 @@ def test_growing_key_norms_move_the_exponent_base():
     parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
 
 
+def test_score_jumps_inside_a_key_block():
+    """Every 128 keys, the last quarter has 16x the norm, so inside one key
+    block a row's scaled score jumps by far more than 2^64 after its first
+    columns were already exponentiated: the band kernel must rescale the
+    probabilities it already holds, and O, in place."""
+    w = workloads.custom("spikes", "bf16", 1, 2, 700, 64, 200, dil=[1, 3], globals_per_b=[[5]], scale=1.0,
+                         seed=39)
+    inp = workloads.make_inputs(w)
+    boost = torch.ones(w.T)
+    boost[torch.arange(w.T) % 128 >= 96] = 16.0
+    inp["k"] = (inp["k"].float() * boost.reshape(1, 1, w.T, 1)).to(torch.bfloat16)
+    parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
+
+
 def test_out_of_range_global_entries_are_ignored_and_flagged():
     w = workloads.custom("bad_g", "bf16", 1, 2, 300, 64, 20, seed=40)
     inp = workloads.make_inputs(w)
