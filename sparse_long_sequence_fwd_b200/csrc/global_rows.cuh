@@ -188,117 +188,255 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
 }
 
 
-// bf16, d = 64: the chunk of K and V is staged in shared memory with
-// coalesced 16-byte loads (K rows padded to 144 bytes so that one thread per
-// key reads its row without bank conflicts); one thread per key forms the
-// scores, and the p*v sums run with 32 column pairs x 8 key groups.
-constexpr int kKsStride = 72;  // bf16 elements per staged K row (64 + 8 pad)
+// bf16, d = 64: tensor-core global rows.  CTA (split, b*h, row group) takes
+// up to 64 global queries of sample b (16 per warp: one m16n8k16 row tile)
+// and cpc consecutive 128-key chunks of the key axis.  Each chunk of K and V
+// is staged once in padded shared memory (cp.async, zero-filled past T);
+// every warp forms S = Q K^T (16 x 128, fp32 in registers), applies the key
+// padding mask, runs the online softmax (log2 domain, exp2) and accumulates
+// O += P V with P re-packed from the S registers as bf16 A fragments and V
+// fragments from ldmatrix.trans.  The partial state (m, l, O) of each row and
+// split goes to the workspace; global_rows_merge_kernel combines the splits.
+// This path is bound by HBM traffic (every K/V row of a (b, h) is read once
+// per row group), not by the tensor rate, so the synchronous warp-level MMA
+// is enough.
+constexpr int kGrKeys = 128;       // keys per chunk
+constexpr int kGrWarps = 4;        // 16 rows per warp
+constexpr int kGrRows = 16 * kGrWarps;
+constexpr int kGrStride = 72;      // bf16 per staged row: 64 + 8 (conflict-free fragments and ldmatrix)
 
-__global__ void __launch_bounds__(kGrThreads) global_rows_bf16_kernel(const __grid_constant__ GlobalRowParams p) {
-    extern __shared__ __align__(16) uint8_t grb_smem[];
-    __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(grb_smem);             // [kChunk][72]
-    __nv_bfloat16* Vs = Ks + kChunk * kKsStride;                                // [kChunk][64]
-    float* qs = reinterpret_cast<float*>(Vs + kChunk * 64);                     // [64]
-    float* ps = qs + 64;                                                         // [kChunk]
-    float* red = ps + kChunk;                                                    // [32]
-    float* accp = red + 32;                                                      // [8][64]
-    __shared__ int is_last;
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t* r, const void* smem_row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(smem_row)));
+}
+// 16-byte global -> shared copy; src_bytes = 0 fills zeros
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
 
-    const int tid = threadIdx.x;
-    const int bh = blockIdx.y;
-    const int b = bh / p.H;
-    const int chunk = blockIdx.x;
-    const int T = p.T;
+__global__ void __launch_bounds__(kGrWarps * 32) global_rows_mma_kernel(const __grid_constant__ GlobalRowParams p) {
+    __shared__ __align__(16) __nv_bfloat16 Ks[kGrKeys * kGrStride];
+    __shared__ __align__(16) __nv_bfloat16 Vs[kGrKeys * kGrStride];
+    __shared__ uint32_t valid_bits[kGrKeys / 32];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;  // fragment row group and column pair
+    const int split = blockIdx.x, bh = blockIdx.y, b = bh / p.H;
     const int nq = p.ws.n_gq[b];
-    if (nq == 0) return;
+    const int row0 = blockIdx.z * kGrRows + warp * 16;  // this warp's first global-row slot
+    if (blockIdx.z * kGrRows >= nq) return;
+    const int T = p.T;
     const size_t base = static_cast<size_t>(bh) * T * 64;
-    const uint4* k4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.k) + base);
-    const uint4* v4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.v) + base);
-    const int j0 = chunk * kChunk;
-    // stage the chunk (8 x 16 B per key and tensor)
-    uint4 kreg[8], vreg[8];
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-        const int u = it * kGrThreads + tid;  // 16-byte unit inside the chunk
-        const int key = u >> 3;
-        const bool in = j0 + key < T;
-        kreg[it] = in ? __ldg(k4 + static_cast<size_t>(j0) * 8 + u) : make_uint4(0u, 0u, 0u, 0u);
-        vreg[it] = in ? __ldg(v4 + static_cast<size_t>(j0) * 8 + u) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-        const int u = it * kGrThreads + tid;
-        const int key = u >> 3, part = u & 7;
-        *reinterpret_cast<uint4*>(Ks + key * kKsStride + part * 8) = kreg[it];
-        *reinterpret_cast<uint4*>(Vs + key * 64 + part * 8) = vreg[it];
-    }
-    const int j = j0 + tid;
-    const bool valid = j < T && !(p.pad && p.pad[static_cast<size_t>(b) * T + j]);
-    const int cp = tid & 31, grp = tid >> 5;  // column pair, key group of 32
-    const int32_t* gq = p.ws.gq_list + static_cast<size_t>(b) * p.gstride;
+    const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(p.k) + base;
+    const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(p.v) + base;
     const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(p.q) + base;
+    const int32_t* gq = p.ws.gq_list + static_cast<size_t>(b) * p.gstride;
+    const bool active = row0 < nq;
 
-    for (int a = 0; a < nq; ++a) {
-        __syncthreads();  // staged chunk visible; previous query's buffers free
-        if (tid < 64) qs[tid] = __bfloat162float(qb[static_cast<size_t>(gq[a]) * 64 + tid]);
-        __syncthreads();
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-        const uint4* krow = reinterpret_cast<const uint4*>(Ks + tid * kKsStride);
+    // Q fragments of rows row0 + g8 and row0 + g8 + 8 (zero past nq)
+    uint32_t qa[4][4];
+    {
+        const int ra = row0 + g8, rb = row0 + g8 + 8;
+        const __nv_bfloat16* qra = ra < nq ? qb + static_cast<size_t>(gq[ra]) * 64 : nullptr;
+        const __nv_bfloat16* qrb = rb < nq ? qb + static_cast<size_t>(gq[rb]) * 64 : nullptr;
 #pragma unroll
-        for (int part = 0; part < 8; ++part) {
-            const uint4 kv = krow[part];
-            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kv);
-            const float2 f0 = __bfloat1622float2(k2[0]), f1 = __bfloat1622float2(k2[1]);
-            const float2 f2 = __bfloat1622float2(k2[2]), f3 = __bfloat1622float2(k2[3]);
-            const float* qq = qs + part * 8;
-            s0 = fmaf(qq[0], f0.x, s0);
-            s1 = fmaf(qq[1], f0.y, s1);
-            s2 = fmaf(qq[2], f1.x, s2);
-            s3 = fmaf(qq[3], f1.y, s3);
-            s0 = fmaf(qq[4], f2.x, s0);
-            s1 = fmaf(qq[5], f2.y, s1);
-            s2 = fmaf(qq[6], f3.x, s2);
-            s3 = fmaf(qq[7], f3.y, s3);
+        for (int ks = 0; ks < 4; ++ks) {
+            const int c0 = 16 * ks + 2 * t4;
+            qa[ks][0] = qra ? *reinterpret_cast<const uint32_t*>(qra + c0) : 0u;
+            qa[ks][1] = qrb ? *reinterpret_cast<const uint32_t*>(qrb + c0) : 0u;
+            qa[ks][2] = qra ? *reinterpret_cast<const uint32_t*>(qra + c0 + 8) : 0u;
+            qa[ks][3] = qrb ? *reinterpret_cast<const uint32_t*>(qrb + c0 + 8) : 0u;
         }
-        const float s = valid ? ((s0 + s1) + (s2 + s3)) * p.sl2 : -INFINITY;
-        const float m = block_reduce_max(s, red);
-        const float m_use = (m == -INFINITY) ? 0.f : m;
-        const float pj = valid ? exp2f(s - m_use) : 0.f;
-        ps[tid] = pj;
-        const float l = block_reduce_sum(pj, red);  // its barriers also publish ps[]
-        float ax = 0.f, ay = 0.f;
-#pragma unroll 8
-        for (int jj = grp * 32; jj < grp * 32 + 32; ++jj) {
-            const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Vs + jj * 64 + 2 * cp));
-            ax = fmaf(ps[jj], vv.x, ax);
-            ay = fmaf(ps[jj], vv.y, ay);
-        }
-        accp[grp * 64 + 2 * cp] = ax;
-        accp[grp * 64 + 2 * cp + 1] = ay;
-        __syncthreads();
-        if (tid < 64) {
-            float t = 0.f;
+    }
+    float o[8][4];
 #pragma unroll
-            for (int gi = 0; gi < 8; ++gi) t += accp[gi * 64 + tid];
-            float* dst = p.ws.partial + ((static_cast<size_t>(bh) * p.gstride + a) * p.nchunk + chunk) * 66;
-            dst[2 + tid] = t;
-            if (tid == 0) {
-                dst[0] = m;
-                dst[1] = l;
+    for (int nd = 0; nd < 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;  // rows g8, g8 + 8
+    const float sl2 = p.sl2;
+
+    const int nblk = (T + kGrKeys - 1) / kGrKeys;
+    const int c_lo = split * p.cpc, c_hi = min(nblk, c_lo + p.cpc);
+    for (int ch = c_lo; ch < c_hi; ++ch) {
+        const int j0 = ch * kGrKeys;
+        __syncthreads();  // previous chunk fully consumed
+        for (int u = tid; u < kGrKeys * 8; u += kGrWarps * 32) {
+            const int key = u >> 3, part = u & 7;
+            const bool in = j0 + key < T;
+            const size_t src = static_cast<size_t>(in ? j0 + key : 0) * 64 + part * 8;
+            cp_async16(Ks + key * kGrStride + part * 8, kb + src, in ? 16u : 0u);
+            cp_async16(Vs + key * kGrStride + part * 8, vb + src, in ? 16u : 0u);
+        }
+        if (tid < kGrKeys) {
+            const int j = j0 + tid;
+            const bool ok = j < T && !(p.pad && p.pad[static_cast<size_t>(b) * T + j]);
+            const uint32_t w = __ballot_sync(0xffffffffu, ok);
+            if (lane == 0) valid_bits[tid >> 5] = w;
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        if (!active) continue;
+
+        // S = Q K^T: 16 key tiles of 8
+        float s[16][4];
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+            const __nv_bfloat16* kr = Ks + (8 * nt + g8) * kGrStride + 2 * t4;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks);
+                const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks + 8);
+                mma_bf16_16816(s[nt], qa[ks], b0, b1);
+            }
+        }
+        // mask, scale, row maxima (each row's 128 scores live in the 4 lanes of its quad)
+        float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const uint32_t vw = valid_bits[nt >> 2] >> ((nt & 3) * 8 + 2 * t4);
+            const bool v0 = vw & 1u, v1 = (vw >> 1) & 1u;
+            s[nt][0] = v0 ? s[nt][0] * sl2 : -INFINITY;
+            s[nt][1] = v1 ? s[nt][1] * sl2 : -INFINITY;
+            s[nt][2] = v0 ? s[nt][2] * sl2 : -INFINITY;
+            s[nt][3] = v1 ? s[nt][3] * sl2 : -INFINITY;
+            mx_a = fmaxf(mx_a, fmaxf(s[nt][0], s[nt][1]));
+            mx_b = fmaxf(mx_b, fmaxf(s[nt][2], s[nt][3]));
+        }
+#pragma unroll
+        for (int off = 1; off <= 2; off <<= 1) {
+            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+        }
+        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+        const float al_a = m_a == -INFINITY ? 0.f : exp2f(m_a - mn_a);
+        const float al_b = m_b == -INFINITY ? 0.f : exp2f(m_b - mn_b);
+        m_a = mn_a;
+        m_b = mn_b;
+        const float bs_a = mn_a == -INFINITY ? 0.f : mn_a, bs_b = mn_b == -INFINITY ? 0.f : mn_b;
+        l_a *= al_a;
+        l_b *= al_b;
+#pragma unroll
+        for (int nd = 0; nd < 8; ++nd) {
+            o[nd][0] *= al_a;
+            o[nd][1] *= al_a;
+            o[nd][2] *= al_b;
+            o[nd][3] *= al_b;
+        }
+        // P (bf16 A fragments) and row sums
+        uint32_t pa[8][4];
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float* sv = s[2 * kk + h];
+                const float e0 = exp2f(sv[0] - bs_a), e1 = exp2f(sv[1] - bs_a);
+                const float e2 = exp2f(sv[2] - bs_b), e3 = exp2f(sv[3] - bs_b);
+                l_a += e0 + e1;
+                l_b += e2 + e3;
+                pa[kk][2 * h] = pack_bf16x2(e0, e1);
+                pa[kk][2 * h + 1] = pack_bf16x2(e2, e3);
+            }
+        }
+        // O += P V: for each 16-key step, two 8-column tiles of V per ldmatrix
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t a[4] = {pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3]};
+#pragma unroll
+            for (int nd = 0; nd < 8; nd += 2) {
+                uint32_t vf[4];
+                ldmatrix_x4_trans(vf, Vs + (16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1)) * kGrStride +
+                                          8 * (nd + (lane >> 4)));
+                mma_bf16_16816(o[nd], a, vf[0], vf[1]);
+                mma_bf16_16816(o[nd + 1], a, vf[2], vf[3]);
             }
         }
     }
-
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) is_last = (atomicAdd(&p.ws.counters[bh], 1) == p.nchunk - 1);
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    merge_partials<__nv_bfloat16>(p, bh, nq, gq, 64);
-    if (tid == 0) p.ws.counters[bh] = 0;
+    if (!active) return;
+    // full row sums over the quad, then the partial state of each row
+#pragma unroll
+    for (int off = 1; off <= 2; off <<= 1) {
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, off);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, off);
+    }
+    const int nsplit = p.nchunk;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int row = row0 + g8 + 8 * h;
+        if (row >= nq) continue;
+        float* dst = p.ws.partial + ((static_cast<size_t>(bh) * p.gstride + row) * nsplit + split) * 66;
+        if (t4 == 0) {
+            dst[0] = h ? m_b : m_a;
+            dst[1] = h ? l_b : l_a;
+        }
+#pragma unroll
+        for (int nd = 0; nd < 8; ++nd) {
+            const int col = 8 * nd + 2 * t4;
+            dst[2 + col] = o[nd][2 * h];
+            dst[3 + col] = o[nd][2 * h + 1];
+        }
+    }
 }
 
-constexpr int kGrBf16Smem = kChunk * kKsStride * 2 + kChunk * 64 * 2 + (64 + kChunk + 32 + 8 * 64) * 4;
+// One CTA per (global-row slot, b*h), one thread per output column: the
+// splits' partial states combine as M = max_c m_c, w_c = 2^(m_c - M),
+// y = sum_c w_c acc_c / sum_c w_c l_c.  The maxima and weights are formed
+// cooperatively (strided over the splits), then every thread streams its
+// column of the partial accumulators with independent loads.
+constexpr int kMaxSplits = 1024;  // the host keeps the split count near 600 CTAs' worth
+__global__ void __launch_bounds__(64) global_rows_merge_kernel(const __grid_constant__ GlobalRowParams p) {
+    __shared__ float wsh[kMaxSplits];
+    __shared__ float red[2];
+    const int a = blockIdx.x, bh = blockIdx.y, b = bh / p.H;
+    if (a >= p.ws.n_gq[b]) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nsplit = p.nchunk;
+    const float* src = p.ws.partial + (static_cast<size_t>(bh) * p.gstride + a) * nsplit * 66;
+
+    float M = -INFINITY;
+    for (int c = tid; c < nsplit; c += 64) M = fmaxf(M, __ldcg(src + static_cast<size_t>(c) * 66));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = fmaxf(red[0], red[1]);
+    const float Mu = M == -INFINITY ? 0.f : M;  // every split empty: all weights 0
+    __syncthreads();
+    float L = 0.f;
+    for (int c = tid; c < nsplit; c += 64) {
+        const float* q = src + static_cast<size_t>(c) * 66;
+        const float w = exp2f(__ldcg(q) - Mu);  // m_c = -inf gives 0
+        wsh[c] = w;
+        L = fmaf(w, __ldcg(q + 1), L);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) red[warp] = L;
+    __syncthreads();
+    L = red[0] + red[1];
+    float acc0 = 0.f, acc1 = 0.f;
+    const float* col = src + 2 + tid;
+    int c = 0;
+#pragma unroll 4
+    for (; c + 1 < nsplit; c += 2) {
+        acc0 = fmaf(wsh[c], __ldcg(col + static_cast<size_t>(c) * 66), acc0);
+        acc1 = fmaf(wsh[c + 1], __ldcg(col + static_cast<size_t>(c + 1) * 66), acc1);
+    }
+    if (c < nsplit) acc0 = fmaf(wsh[c], __ldcg(col + static_cast<size_t>(c) * 66), acc0);
+    const float y = L > 0.f ? (acc0 + acc1) / L : 0.f;
+    const int32_t g = p.ws.gq_list[static_cast<size_t>(b) * p.gstride + a];
+    reinterpret_cast<__nv_bfloat16*>(p.out)[(static_cast<size_t>(bh) * p.T + g) * 64 + tid] = __float2bfloat16_rn(y);
+}
 
 }  // namespace lf

@@ -47,14 +47,24 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
     size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, total;
-    int W, gstride, nchunk, ngp;
+    int W, gstride, nchunk, ngp, cpc;  // nchunk: partial states per global row
 };
 
 Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
     Layout L{};
     L.W = (T + 31) / 32;
     L.gstride = std::max(1, std::min(n_global, T));
-    L.nchunk = (T + kChunk - 1) / kChunk;
+    if (dtype == LF_BF16) {
+        // tensor-core global rows: 128-key chunks, cpc per CTA, about 600 CTAs in all
+        const int nblk = (T + kGrKeys - 1) / kGrKeys;
+        const long units = long(nblk) * B * H * ((L.gstride + kGrRows - 1) / kGrRows);
+        L.cpc = static_cast<int>(std::max(1L, std::min<long>(nblk, units / 600)));
+        L.nchunk = (nblk + L.cpc - 1) / L.cpc;
+        while (L.nchunk > kMaxSplits) L.nchunk = (nblk + ++L.cpc - 1) / L.cpc;
+    } else {
+        L.cpc = 1;
+        L.nchunk = (T + kChunk - 1) / kChunk;
+    }
     L.ngp = (L.gstride + 15) & ~15;
     size_t o = 0;
     L.off_ngq = o; o = align256(o + sizeof(int32_t) * B);
@@ -96,8 +106,6 @@ lf_status set_kernel_attributes() {
         cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
             cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(global_rows_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrBf16Smem) !=
             cudaSuccess)
         return LF_ERR_CUDA;
     return LF_OK;
@@ -346,14 +354,22 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         gp.gstride = L.gstride;
         gp.nchunk = L.nchunk;
         gp.sl2 = sl2;
-        const dim3 grid(L.nchunk, B * H);
-        const int DP = d <= 32 ? 32 : (d <= 64 ? 64 : 128);
-        const size_t smem = size_t(kChunk * DP + DP + kChunk + 32 + kGrThreads) * 4;
-        if (dtype == LF_BF16) global_rows_bf16_kernel<<<grid, kGrThreads, kGrBf16Smem, stream>>>(gp);
-        else if (DP == 32) global_rows_kernel<float, 32><<<grid, kGrThreads, smem, stream>>>(gp);
-        else if (DP == 64) global_rows_kernel<float, 64><<<grid, kGrThreads, smem, stream>>>(gp);
-        else global_rows_kernel<float, 128><<<grid, kGrThreads, smem, stream>>>(gp);
-        ++launches;
+        gp.cpc = L.cpc;
+        if (dtype == LF_BF16) {
+            // key splits x (b, h) x groups of 64 global rows, then the merge of the splits
+            global_rows_mma_kernel<<<dim3(L.nchunk, B * H, (L.gstride + kGrRows - 1) / kGrRows), kGrWarps * 32, 0,
+                                     stream>>>(gp);
+            global_rows_merge_kernel<<<dim3(L.gstride, B * H), 64, 0, stream>>>(gp);
+            launches += 2;
+        } else {
+            const dim3 grid(L.nchunk, B * H);
+            const int DP = d <= 32 ? 32 : (d <= 64 ? 64 : 128);
+            const size_t smem = size_t(kChunk * DP + DP + kChunk + 32 + kGrThreads) * 4;
+            if (DP == 32) global_rows_kernel<float, 32><<<grid, kGrThreads, smem, stream>>>(gp);
+            else if (DP == 64) global_rows_kernel<float, 64><<<grid, kGrThreads, smem, stream>>>(gp);
+            else global_rows_kernel<float, 128><<<grid, kGrThreads, smem, stream>>>(gp);
+            ++launches;
+        }
     }
     if (cudaGetLastError() != cudaSuccess) return LF_ERR_CUDA;
     t_last_launches = launches;

@@ -26,7 +26,7 @@ struct Workspace {
     int32_t* gk_list;   // [B][gstride] sorted
     uint32_t* gbit;     // [B][W]   bit i = position i is a global query
     int32_t* counters;  // [B*H]    arrival tickets of the global-row kernel (kept at 0 between calls)
-    float* partial;     // [B*H][gstride][nchunk][d + 2]
+    float* partial;     // [B*H][gstride][nchunk][d + 2] partial (m, l, acc) of each global row
     __nv_bfloat16* kg;  // [B*H][ngp][64] packed global keys (bf16 path)
     __nv_bfloat16* vg;  // [B*H][ngp][64] packed global values
 };
@@ -49,7 +49,8 @@ struct GlobalRowParams {
     void* out;
     const uint8_t* pad;
     Workspace ws;
-    int B, H, T, d, gstride, nchunk;
+    int B, H, T, d, gstride, nchunk;  // nchunk: partial states per global row
+    int cpc;                          // bf16: 128-key chunks per CTA
     float sl2;  // scale * log2(e)
 };
 

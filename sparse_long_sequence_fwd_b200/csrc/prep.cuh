@@ -20,19 +20,29 @@ namespace lf {
 
 constexpr int kPrepThreads = 256;
 
+// Exclusive prefix sum of v over the CTA (warp shuffles, then the warps'
+// totals); sbuf holds at least kPrepThreads / 32 ints.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* sbuf) {
-    // sbuf: kPrepThreads ints; returns exclusive prefix, leaves the total in sbuf[kPrepThreads-1] + v_last
-    const int tid = threadIdx.x;
-    sbuf[tid] = v;
-    __syncthreads();
-    for (int off = 1; off < kPrepThreads; off <<= 1) {
-        int t = tid >= off ? sbuf[tid - off] : 0;
-        __syncthreads();
-        sbuf[tid] += t;
-        __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
     }
-    int incl = sbuf[tid];
-    return incl - v;
+    if (lane == 31) sbuf[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int t = lane < kPrepThreads / 32 ? sbuf[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < kPrepThreads / 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        if (lane < kPrepThreads / 32) sbuf[lane] = t;
+    }
+    __syncthreads();
+    return (warp ? sbuf[warp - 1] : 0) + x - v;
 }
 
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {

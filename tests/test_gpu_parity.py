@@ -116,6 +116,14 @@ def test_growing_key_norms_move_the_exponent_base():
     parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
 
 
+def test_many_global_rows_span_several_row_groups():
+    """150 global queries of one sample (three groups of 64 rows in the
+    global-row kernel), padding after position 1200, every element checked."""
+    w = workloads.custom("many_g", "bf16", 1, 2, 1500, 64, 60, n_random_globals=150, pad_from=[1200], seed=42)
+    inp = workloads.make_inputs(w)
+    parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
+
+
 def test_score_jumps_inside_a_key_block():
     """Every 128 keys, the last quarter has 16x the norm, so inside one key
     block a row's scaled score jumps by far more than 2^64 after its first
@@ -146,11 +154,12 @@ def test_out_of_range_global_entries_are_ignored_and_flagged():
     assert st == 0 and flags == 0
 
 
-def test_deterministic_and_three_launches():
+def test_deterministic_and_four_launches():
+    """prep, band, global rows, merge of the global rows' key splits."""
     w = workloads.BASE
     inp = workloads.make_inputs(w)
     a = parity.run_gpu(w, inp)
-    assert lf_attn.last_launch_count() == 3
+    assert lf_attn.last_launch_count() == 4
     b = parity.run_gpu(w, inp)
     assert torch.equal(a, b)
 

@@ -59,7 +59,7 @@ def test_static_matches_allocating_entry_point_twice(w):
 
 
 def test_sizes_beyond_the_scratch_are_rejected_before_launch():
-    B, H, T, d, ng = 1, 16, 16384, 64, 256
+    B, H, T, d, ng = 1, 16, 16384, 64, 4096
     need = lf_attn.workspace_bytes(B, H, T, d, ng, lf_attn.LF_BF16)
     assert need > SCRATCH_LIMIT
     q = torch.zeros(B, H, T, d, dtype=torch.bfloat16, device="cuda")
