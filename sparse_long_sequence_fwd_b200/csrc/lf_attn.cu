@@ -36,6 +36,11 @@ struct DeviceState {
     size_t ws_bytes = 0;
     void* io = nullptr;  // staging for lf_attn_fwd_host
     size_t io_bytes = 0;
+    // The global-row kernels run on a low-priority side stream forked after
+    // prep, so their CTAs fill the SMs the band kernel's CTAs leave as they
+    // finish; null: everything runs in order on the caller's stream.
+    cudaStream_t aux = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 };
 
 std::mutex g_mu;
@@ -123,6 +128,12 @@ lf_status device_state(DeviceState** out) {
         if (cudaMalloc(&s.status, 256) != cudaSuccess) return LF_ERR_NO_MEMORY;
         if (cudaMemset(s.status, 0, 256) != cudaSuccess) return LF_ERR_CUDA;
         if (set_kernel_attributes() != LF_OK) return LF_ERR_CUDA;
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&s.aux, cudaStreamNonBlocking, least) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s.ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s.ev_join, cudaEventDisableTiming) != cudaSuccess)
+            return LF_ERR_CUDA;
         s.init = true;
     }
     *out = &s;
@@ -249,6 +260,12 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         prep_kernel<<<B * H, kPrepThreads, prep_smem, stream>>>(pp);
         ++launches;
     }
+    // The global rows depend on prep only: with a side stream they are forked
+    // here and joined after the band kernel, which is launched first and so
+    // takes the SMs first.
+    const bool global_stage = n_global > 0 && (stages & 4u);
+    const bool fork = global_stage && (stages & 2u) && dtype == LF_BF16 && ds->aux != nullptr;
+    if (fork && cudaEventRecord(ds->ev_fork, stream) != cudaSuccess) return LF_ERR_CUDA;
 
     if (!(stages & 2u)) {
         // band stage skipped
@@ -341,7 +358,12 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         ++launches;
     }
 
-    if (n_global > 0 && (stages & 4u)) {
+    if (global_stage) {
+        cudaStream_t gs = stream;
+        if (fork) {
+            if (cudaStreamWaitEvent(ds->aux, ds->ev_fork, 0) != cudaSuccess) return LF_ERR_CUDA;
+            gs = ds->aux;
+        }
         // K2: rows of the global queries
         GlobalRowParams gp;
         gp.q = q;
@@ -358,8 +380,8 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         if (dtype == LF_BF16) {
             // key splits x (b, h) x groups of 64 global rows, then the merge of the splits
             global_rows_mma_kernel<<<dim3(L.nchunk, B * H, (L.gstride + kGrRows - 1) / kGrRows), kGrWarps * 32, 0,
-                                     stream>>>(gp);
-            global_rows_merge_kernel<<<dim3(L.gstride, B * H), 64, 0, stream>>>(gp);
+                                     gs>>>(gp);
+            global_rows_merge_kernel<<<dim3(L.gstride, B * H), 64, 0, gs>>>(gp);
             launches += 2;
         } else {
             const dim3 grid(L.nchunk, B * H);
@@ -370,6 +392,9 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
             else global_rows_kernel<float, 128><<<grid, kGrThreads, smem, stream>>>(gp);
             ++launches;
         }
+        if (fork && (cudaEventRecord(ds->ev_join, ds->aux) != cudaSuccess ||
+                     cudaStreamWaitEvent(stream, ds->ev_join, 0) != cudaSuccess))
+            return LF_ERR_CUDA;
     }
     if (cudaGetLastError() != cudaSuccess) return LF_ERR_CUDA;
     t_last_launches = launches;
