@@ -76,6 +76,11 @@ typedef enum {
  *   stream      a cudaStream_t (NULL = legacy default stream)
  *
  * Returns LF_OK once the kernels are queued; nothing is synchronised.
+ * On the bf16 path with global tokens, the global-row kernels are queued on
+ * a library-owned low-priority stream that waits for the earlier work of
+ * `stream` and that `stream` waits for in turn, so the call stays ordered
+ * on `stream` (also under stream capture).  Calls on different streams
+ * share that side stream, so their global-row kernels run in call order.
  */
 lf_status lf_attn_fwd(const void* q, const void* k, const void* v, void* out,
                       int B, int H, int T, int d, int r, const int32_t* dil,
