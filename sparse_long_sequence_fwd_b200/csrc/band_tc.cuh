@@ -65,7 +65,12 @@ constexpr int kBarQFull = 0, kBarQEmpty = kBarQFull + kStages, kBarKFull = kBarQ
               kBarKEmpty = kBarKFull + kStages, kBarVFull = kBarKEmpty + kStages, kBarVEmpty = kBarVFull + kStages,
               kBarSFull = kBarVEmpty + kStages, kBarSFree = kBarSFull + 1, kBarPFull = kBarSFree + 1,
               kBarOFull = kBarPFull + 1, kBarDrain = kBarOFull + 1, kNumBars = kBarDrain + 1;
-constexpr int kOffMisc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
+// Tile descriptors (BandTile), one per Q slot: written by the producer before
+// it arrives on the slot's Q-full barrier, read by the MMA and softmax roles
+// after waiting on it, so only the producer decodes work items.
+constexpr int kOffDesc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
+constexpr int kDescBytes = 64;
+constexpr int kOffMisc = kOffDesc + kStages * kDescBytes;
 constexpr int kMiscBytes = 16;
 constexpr int kBandSmem = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 static_assert(kBandCtasPerSm * (kBandSmem + 1024) <= 233472, "shared memory budget for two CTAs per SM");
@@ -79,6 +84,7 @@ struct BandTile {
     int b, bh, c, dil, dk, R;
     int Tc, q0, kbase, kb_lo, nbb, ngk, ngb;
 };
+static_assert(sizeof(BandTile) <= kDescBytes, "tile descriptor slot");
 
 // Out of line: every role walks the same tiles, and one copy of this code
 // (integer divisions included) keeps the kernel small.
@@ -180,6 +186,7 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
         if (kc.blk == 0) {
             const uint32_t qs = qt & 1u;
             if (!mbar_wait(&bars[kBarQEmpty + qs], ((qt >> 1) & 1u) ^ 1u, abort_flag)) return false;
+            *reinterpret_cast<BandTile*>(smem + kOffDesc + qs * kDescBytes) = t;  // released by the arrive
             mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes);
             uint8_t* dQ = smem + kOffQ + qs * kTileBytes;
             for (int u = 0; u < kBM; u += t.R)
@@ -279,26 +286,30 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
         return true;
     };
 
-    BlockCursor c;
-    c.start(p);
-    uint32_t g = 0, qt = 0;
+    uint32_t g = 0, qt = 0, qs = 0;
+    int item = blockIdx.x, blk = 0, nb = 0, nbb = 0, ngk = 0;
     int prev_nk = 0;
     bool prev_first = false;
     for (;;) {  // S(g), then the product of block g - 1
-        const bool have = c.valid(p);
+        const bool have = item < p.n_items;
+        int cur_nk = 0;
+        bool cur_first = false;
         if (have) {
-            const BandTile& t = c.t;
-            const uint32_t qs = (qt - (c.blk == 0 ? 0u : 1u)) & 1u;
-            if (c.blk == 0) {
+            if (blk == 0) {  // the tile's Q has landed and its descriptor is visible
+                qs = qt & 1u;
                 if (!mbar_wait(&bars[kBarQFull + qs], (qt >> 1) & 1u, abort_flag)) break;
                 ++qt;
+                const BandTile* d = reinterpret_cast<const BandTile*>(smem + kOffDesc + qs * kDescBytes);
+                nbb = d->nbb;
+                ngk = d->ngk;
+                nb = nbb + d->ngb;
             }
             const uint32_t s = g & 1u;
             if (!mbar_wait(&bars[kBarKFull + s], (g >> 1) & 1u, abort_flag) ||
                 (g > 0 && !mbar_wait(&bars[kBarSFree], (g - 1) & 1u, abort_flag)))
                 break;
             tc_fence_after();
-            const int ncols = c.blk < t.nbb ? kBN : global_block_cols(t.ngk, c.blk - t.nbb);
+            const int ncols = blk < nbb ? kBN : global_block_cols(ngk, blk - nbb);
             const uint32_t ids = ncols == kBN ? idesc_s : idesc_bf16(kBM, ncols, 0, 0);
             const uint64_t dq = dQ[qs], dk = dK[s];
             tc_mma<false>(tS, dq + 0, dk + 0, ids);  // K-steps of 16 (32 bytes = 2 units)
@@ -307,14 +318,19 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
             tc_mma<true>(tS, dq + 6, dk + 6, ids);
             tc_commit(&bars[kBarSFull]);
             tc_commit(&bars[kBarKEmpty + s]);
-            if (c.blk == c.nb - 1) tc_commit(&bars[kBarQEmpty + qs]);
+            if (blk == nb - 1) tc_commit(&bars[kBarQEmpty + qs]);
+            cur_nk = ncols;
+            cur_first = blk == 0;
         }
         if (g > 0 && !issue_pv(g - 1, prev_nk, prev_first)) break;
         if (!have) break;
-        prev_nk = c.blk < c.t.nbb ? kBN : global_block_cols(c.t.ngk, c.blk - c.t.nbb);
-        prev_first = c.blk == 0;
+        prev_nk = cur_nk;
+        prev_first = cur_first;
         ++g;
-        c.next(p);
+        if (++blk == nb) {
+            blk = 0;
+            item += gridDim.x;
+        }
     }
     tc_commit(&bars[kBarDrain]);
 }
@@ -379,8 +395,8 @@ __device__ __forceinline__ uint32_t pick4(const uint32_t* v, int c) {
     return c == 0 ? v[0] : (c == 1 ? v[1] : (c == 2 ? v[2] : v[3]));
 }
 
-__device__ __forceinline__ void softmax_role(const BandTcParams& p, uint64_t* bars, volatile int* abort_flag,
-                                             uint32_t tmem_base) {
+__device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
+                                             volatile int* abort_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wq = warp & 3;
     const int x = wq * 32 + lane;  // query row inside the tile = TMEM lane
@@ -431,12 +447,17 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint64_t* ba
         }
     };
 
+    uint32_t qt = 0;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-        const BandTile t = band_decode(p, item);
+        // the tile's descriptor, published by the producer with its Q tile
+        const uint32_t qs = qt & 1u;
+        if (!wait_warp(&bars[kBarQFull + qs], (qt >> 1) & 1u)) return;
+        ++qt;
+        const BandTile t = *reinterpret_cast<const BandTile*>(smem + kOffDesc + qs * kDescBytes);
         const int ip = t.q0 + x;         // decimated row index
         const int i = t.c + t.dil * ip;  // position in the sequence
-        bool row_ok = ip < t.Tc;
-        if (row_ok && ((p.gbit[static_cast<size_t>(t.b) * p.W + (i >> 5)] >> (i & 31)) & 1u)) row_ok = false;
+        // global-row bitmap word of this row; consumed only when the tile's rows are written
+        const uint32_t gbw = ip < t.Tc ? __ldg(p.gbit + static_cast<size_t>(t.b) * p.W + (i >> 5)) : 0u;
         const int32_t* gk = p.gk_list + static_cast<size_t>(t.b) * p.gstride;
         const int reach = t.dil * p.r;
         // the first block of global keys, one key per lane and chunk, fetched early
@@ -615,7 +636,7 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint64_t* ba
         }
         // ---- this tile's rows: y = O / l, written once its last product is done
         pend = true;
-        pend_ok = row_ok;
+        pend_ok = ip < t.Tc && !((gbw >> (i & 31)) & 1u);
         pend_inv = l_row > 0.f ? 1.f / l_row : 0.f;
         pend_dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t.bh) * p.T + i) * kHD);
     }
@@ -677,7 +698,7 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
     } else if (warp == 1) {
         if (lane == 0) mma_role(p, smem, bars, abort_flag, tmem_base);
     } else {
-        softmax_role(p, bars, abort_flag, tmem_base);
+        softmax_role(p, smem, bars, abort_flag, tmem_base);
     }
 
     tc_fence_before();
