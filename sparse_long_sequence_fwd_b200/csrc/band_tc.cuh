@@ -370,7 +370,7 @@ __device__ __forceinline__ void rescale_p_chunks(uint32_t tP, int nchunks, float
 }
 
 // Multiplies this thread's row of O (64 fp32 columns) by alpha, in TMEM.
-__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+__device__ __noinline__ void rescale_o(uint32_t tO, float alpha) {
 #pragma unroll 1
     for (int part = 0; part < 4; ++part) {
         uint32_t orr[16];
@@ -382,13 +382,35 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
     }
 }
 
-// Multiplies 16 packed bf16 pairs by alpha.
-__device__ __forceinline__ void scale_packed(uint32_t* pk, float alpha) {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pk[u]));
-        pk[u] = pack_bf16x2(f.x * alpha, f.y * alpha);
+// Writes this thread's output row, y = O * inv as bf16 (dst null: row not
+// written), from TMEM.  Once per tile, out of line.
+__device__ __noinline__ void write_rows(uint32_t tO, uint4* dst, float inv) {
+#pragma unroll 1
+    for (int part = 0; part < 4; ++part) {
+        uint32_t o[16];
+        tmem_ld16(tO + 16u * part, o);
+        tmem_ld_wait16(o);
+        if (dst) {
+            uint4 v0, v1;
+            v0.x = pack_bf16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+            v0.y = pack_bf16x2(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+            v0.z = pack_bf16x2(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+            v0.w = pack_bf16x2(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+            v1.x = pack_bf16x2(__uint_as_float(o[8]) * inv, __uint_as_float(o[9]) * inv);
+            v1.y = pack_bf16x2(__uint_as_float(o[10]) * inv, __uint_as_float(o[11]) * inv);
+            v1.z = pack_bf16x2(__uint_as_float(o[12]) * inv, __uint_as_float(o[13]) * inv);
+            v1.w = pack_bf16x2(__uint_as_float(o[14]) * inv, __uint_as_float(o[15]) * inv);
+            dst[2 * part] = v0;
+            dst[2 * part + 1] = v1;
+        }
     }
+}
+
+// Rare path of a score jump inside a block: multiplies the first nchunks P
+// chunks of this thread's row, and (with_o) its row of O, by alpha, in TMEM.
+__device__ __noinline__ void rescale_held(uint32_t tP, int nchunks, uint32_t tO, bool with_o, float alpha) {
+    rescale_p_chunks(tP, nchunks, alpha);
+    if (with_o) rescale_o(tO, alpha);
 }
 
 __device__ __forceinline__ uint32_t pick4(const uint32_t* v, int c) {
@@ -426,25 +448,7 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     auto flush = [&]() {
         if (!pend) return;
         pend = false;
-#pragma unroll 1
-        for (int part = 0; part < 4; ++part) {
-            uint32_t o[16];
-            tmem_ld16(tO + 16u * part, o);
-            tmem_ld_wait16(o);
-            if (pend_ok) {
-                uint4 v0, v1;
-                v0.x = pack_bf16x2(__uint_as_float(o[0]) * pend_inv, __uint_as_float(o[1]) * pend_inv);
-                v0.y = pack_bf16x2(__uint_as_float(o[2]) * pend_inv, __uint_as_float(o[3]) * pend_inv);
-                v0.z = pack_bf16x2(__uint_as_float(o[4]) * pend_inv, __uint_as_float(o[5]) * pend_inv);
-                v0.w = pack_bf16x2(__uint_as_float(o[6]) * pend_inv, __uint_as_float(o[7]) * pend_inv);
-                v1.x = pack_bf16x2(__uint_as_float(o[8]) * pend_inv, __uint_as_float(o[9]) * pend_inv);
-                v1.y = pack_bf16x2(__uint_as_float(o[10]) * pend_inv, __uint_as_float(o[11]) * pend_inv);
-                v1.z = pack_bf16x2(__uint_as_float(o[12]) * pend_inv, __uint_as_float(o[13]) * pend_inv);
-                v1.w = pack_bf16x2(__uint_as_float(o[14]) * pend_inv, __uint_as_float(o[15]) * pend_inv);
-                pend_dst[2 * part] = v0;
-                pend_dst[2 * part + 1] = v1;
-            }
-        }
+        write_rows(tO, pend_ok ? pend_dst : nullptr, pend_inv);
     };
 
     uint32_t qt = 0;
@@ -529,16 +533,16 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
 
             if (!wait_warp(&bars[kBarSFull], g & 1u)) return;
             tc_fence_after();
-            uint32_t sa[32], sb[32], pka[16], pkb[16];
-            tmem_ld32(tS, sa);
+            if (!ensure_p_ready()) return;
             float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-            // chunk c of the block: scores in cur (the next chunk loads into nxt), P into pk;
-            // P of chunk c - 1 (in pk_prev) is stored one chunk late
-            auto chunk = [&](uint32_t* cur, uint32_t* nxt, uint32_t* pk, uint32_t* pk_prev, const int c) -> bool {
+            // one body for every chunk: a second copy (for a load in flight during the
+            // previous chunk) costs more in instruction fetch than it hides
+#pragma unroll 1
+            for (int c = 0; c < nch; ++c) {
+                uint32_t cur[32];
+                tmem_ld32(tS + 32u * c, cur);
                 tmem_ld_wait(cur);
-                if (c + 1 < nch) {
-                    tmem_ld32(tS + 32u * (c + 1), nxt);
-                } else {  // the whole S block is in registers or consumed: the MMA may overwrite it
+                if (c + 1 == nch) {  // the whole S block has been read: the MMA may overwrite it
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars[kBarSFree]);
@@ -600,14 +604,10 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                         lsum[2] *= alpha;
                         lsum[3] *= alpha;
                     }
-                    if (c > 0) scale_packed(pk_prev, alpha);
-                    if (c > 1) rescale_p_chunks(tP, c - 1, alpha);
-                    if (blk > 0) {
-                        if (!ensure_p_ready()) return false;
-                        rescale_o(tO, alpha);
-                    }
+                    if (c > 0 || blk > 0) rescale_held(tP, c, tO, blk > 0, alpha);
                 }
                 const float nb2 = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
                     const float e0 = ex2_approx(fmaf(__uint_as_float(cur[j]), kmul, nb2));
@@ -615,19 +615,8 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                     lsum[(j >> 1) & 3] += e0 + e1;
                     pk[j >> 1] = pack_bf16x2(e0, e1);
                 }
-                if (c > 0) {
-                    if (!ensure_p_ready()) return false;
-                    tmem_st16(tP + 16u * (c - 1), pk_prev);
-                }
-                return true;
-            };
-#pragma unroll 1
-            for (int c = 0; c < nch; c += 2) {
-                if (!chunk(sa, sb, pka, pkb, c)) return;
-                if (c + 1 < nch && !chunk(sb, sa, pkb, pka, c + 1)) return;
+                tmem_st16(tP + 16u * c, pk);
             }
-            if (!ensure_p_ready()) return;
-            tmem_st16(tP + 16u * (nch - 1), (nch & 1) ? pka : pkb);
             l_row += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
             tmem_st_wait();
             tc_fence_before();
