@@ -681,6 +681,8 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the set-up above may overlap the prep kernel; its lists and packed keys are read below
+    grid_dep_wait();
 
     if (warp == 0) {
         if (lane == 0) producer_role(p, smem, bars, abort_flag);

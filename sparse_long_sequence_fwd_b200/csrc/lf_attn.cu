@@ -354,7 +354,19 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         bp.items_per_b = items_per_b;
         bp.n_items = items_per_b * B;
         const int grid = std::min(bp.n_items, kBandCtasPerSm * ds->sm_count);
-        band_tc_kernel<<<grid, kBandThreads, kBandSmem, stream>>>(bp);
+        // right after prep on the same stream, launched as its programmatic dependent: the
+        // band kernel's set-up (barriers, TMEM, tensor-map prefetch) overlaps prep
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(kBandThreads);
+        cfg.dynamicSmemBytes = kBandSmem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = (stages & 1u) ? 1 : 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, band_tc_kernel, bp) != cudaSuccess) return LF_ERR_CUDA;
         ++launches;
     }
 

@@ -15,6 +15,7 @@
 // beyond the list, so the band kernel can stage them with one TMA box.
 #pragma once
 #include "lf_common.cuh"
+#include "ptx.cuh"
 
 namespace lf {
 
@@ -53,6 +54,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     int* gk_s = scan_k + kPrepThreads;                               // [gstride]
     __shared__ int n_k_total;
 
+    grid_dep_launch();  // the band kernel may set itself up meanwhile; it waits for this grid before reading
     const int tid = threadIdx.x;
     const int b = blockIdx.x / p.H;
     const int h = blockIdx.x - b * p.H;
