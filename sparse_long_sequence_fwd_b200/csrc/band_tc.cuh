@@ -564,9 +564,11 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                             m |= in_window ? 0u : (1u << a);
                         }
                     }
+                    if (!__all_sync(0xffffffffu, m == 0xffffffffu)) {  // only chunks some row masks
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (!((m >> j) & 1u)) cur[j] = fill;
+                        for (int j = 0; j < 32; ++j)
+                            if (!((m >> j) & 1u)) cur[j] = fill;
+                    }
                 }
                 float mx;
                 if (pos) {
