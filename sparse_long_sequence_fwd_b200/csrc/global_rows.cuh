@@ -222,9 +222,10 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most N committed groups of this thread are still in flight
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __global__ void __launch_bounds__(kGrWarps * 32) global_rows_mma_kernel(const __grid_constant__ GlobalRowParams p) {
     __shared__ __align__(16) __nv_bfloat16 Ks[kGrKeys * kGrStride];
@@ -271,22 +272,31 @@ __global__ void __launch_bounds__(kGrWarps * 32) global_rows_mma_kernel(const __
     for (int ch = c_lo; ch < c_hi; ++ch) {
         const int j0 = ch * kGrKeys;
         __syncthreads();  // previous chunk fully consumed
+        // K, then V, as two groups: S and the softmax run while V is still arriving
         for (int u = tid; u < kGrKeys * 8; u += kGrWarps * 32) {
             const int key = u >> 3, part = u & 7;
             const bool in = j0 + key < T;
             const size_t src = static_cast<size_t>(in ? j0 + key : 0) * 64 + part * 8;
             cp_async16(Ks + key * kGrStride + part * 8, kb + src, in ? 16u : 0u);
+        }
+        cp_async_commit();
+        for (int u = tid; u < kGrKeys * 8; u += kGrWarps * 32) {
+            const int key = u >> 3, part = u & 7;
+            const bool in = j0 + key < T;
+            const size_t src = static_cast<size_t>(in ? j0 + key : 0) * 64 + part * 8;
             cp_async16(Vs + key * kGrStride + part * 8, vb + src, in ? 16u : 0u);
         }
+        cp_async_commit();
         if (tid < kGrKeys) {
             const int j = j0 + tid;
             const bool ok = j < T && !(p.pad && p.pad[static_cast<size_t>(b) * T + j]);
             const uint32_t w = __ballot_sync(0xffffffffu, ok);
             if (lane == 0) valid_bits[tid >> 5] = w;
         }
-        cp_async_wait_all();
+        cp_async_wait<1>();  // K has landed
         __syncthreads();
-        if (!active) continue;
+        uint32_t pa[8][4];  // P of this warp's rows as bf16 A fragments
+        if (active) {
 
         // S = Q K^T: 16 key tiles of 8
         float s[16][4];
@@ -335,7 +345,6 @@ __global__ void __launch_bounds__(kGrWarps * 32) global_rows_mma_kernel(const __
             o[nd][3] *= al_b;
         }
         // P (bf16 A fragments) and row sums
-        uint32_t pa[8][4];
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
@@ -349,6 +358,10 @@ __global__ void __launch_bounds__(kGrWarps * 32) global_rows_mma_kernel(const __
                 pa[kk][2 * h + 1] = pack_bf16x2(e2, e3);
             }
         }
+        }
+        cp_async_wait<0>();  // V has landed
+        __syncthreads();
+        if (!active) continue;
         // O += P V: for each 16-key step, two 8-column tiles of V per ldmatrix
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
