@@ -146,7 +146,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// Walks the (item, block) sequence of this CTA in the order every role uses.
+// Work item of a slot: the CTA with blockIdx b takes slots b, b + grid, ...;
+// the host may order the items so the longest tiles come first.
+__device__ __forceinline__ int slot_item(const BandTcParams& p, int slot) {
+    return p.item_order ? __ldg(p.item_order + slot) : slot;
+}
+
+// Walks the (slot, block) sequence of this CTA in the order every role uses.
 struct BlockCursor {
     int item, blk, nb;
     BandTile t;
@@ -154,7 +160,7 @@ struct BlockCursor {
         item = blockIdx.x;
         blk = 0;
         if (item < p.n_items) {
-            t = band_decode(p, item);
+            t = band_decode(p, slot_item(p, item));
             nb = t.nbb + t.ngb;
         } else {
             nb = 0;
@@ -166,7 +172,7 @@ struct BlockCursor {
         blk = 0;
         item += gridDim.x;
         if (item < p.n_items) {
-            t = band_decode(p, item);
+            t = band_decode(p, slot_item(p, item));
             nb = t.nbb + t.ngb;
         }
     }

@@ -41,6 +41,13 @@ struct DeviceState {
     // finish; null: everything runs in order on the caller's stream.
     cudaStream_t aux = nullptr;
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    // Band work items in longest-first order (device copy), for the shape in
+    // order_key; rebuilt outside stream capture when the shape changes.
+    bool may_order = true;  // false: never allocate for it (the allocation-free entry point)
+    int32_t* order = nullptr;
+    size_t order_cap = 0;
+    bool order_identity = true;
+    std::vector<int> order_key;
 };
 
 std::mutex g_mu;
@@ -353,6 +360,46 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         bp.sl2 = sl2;
         bp.items_per_b = items_per_b;
         bp.n_items = items_per_b * B;
+        bp.item_order = nullptr;
+        if (ds->may_order) {
+            // Longest tiles first: with fewer CTAs than tiles, the CTAs that take a second
+            // tile then take one of the short tiles at the sequence ends.
+            std::vector<int> key = {B, H, T, r_eff};
+            for (int h = 0; h < H; ++h) key.push_back(dil ? dil[h] : 1);
+            if (key != ds->order_key && !is_capturing(stream)) {
+                std::vector<int> cost;
+                cost.reserve(bp.n_items);
+                for (int b = 0; b < B; ++b)
+                    for (int h = 0; h < H; ++h) {
+                        const int dl = bp.dk_dil[kind_of_head[h]];
+                        for (int c = 0; c < dl; ++c) {
+                            const int Tc = (T - c + dl - 1) / dl;
+                            for (int q0 = 0; q0 < Tc; q0 += kBM) {
+                                const int kbase = q0 - r_eff;
+                                const int lo = std::max(0, kbase), hi = std::min(Tc - 1, q0 + kBM - 1 + r_eff);
+                                cost.push_back((hi - kbase) / kBN + 1 - (lo - kbase) / kBN);
+                            }
+                        }
+                    }
+                std::vector<int32_t> order(cost.size());
+                for (size_t a = 0; a < order.size(); ++a) order[a] = static_cast<int32_t>(a);
+                std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) { return cost[x] > cost[y]; });
+                bool identity = true;
+                for (size_t a = 0; a < order.size() && identity; ++a) identity = order[a] == static_cast<int32_t>(a);
+                if (!identity) {
+                    void* buf = ds->order;
+                    if ((st = grow(&buf, &ds->order_cap, order.size() * sizeof(int32_t), stream)) != LF_OK) return st;
+                    ds->order = static_cast<int32_t*>(buf);
+                    // from pageable memory: returns once the data is staged, ordered on the stream
+                    if (cudaMemcpyAsync(ds->order, order.data(), order.size() * sizeof(int32_t),
+                                        cudaMemcpyHostToDevice, stream) != cudaSuccess)
+                        return LF_ERR_CUDA;
+                }
+                ds->order_identity = identity;
+                ds->order_key = key;
+            }
+            if (key == ds->order_key && !ds->order_identity) bp.item_order = ds->order;
+        }
         const int grid = std::min(bp.n_items, kBandCtasPerSm * ds->sm_count);
         // right after prep on the same stream, launched as its programmatic dependent: the
         // band kernel's set-up (barriers, TMEM, tensor-map prefetch) overlaps prep
@@ -559,7 +606,11 @@ void lf_attn_release(void) {
         cudaSetDevice(dev);
         if (s.ws) cudaFree(s.ws);
         if (s.io) cudaFree(s.io);
+        if (s.order) cudaFree(s.order);
         if (s.status) cudaFree(s.status);
+        if (s.ev_fork) cudaEventDestroy(s.ev_fork);
+        if (s.ev_join) cudaEventDestroy(s.ev_join);
+        if (s.aux) cudaStreamDestroy(s.aux);
         s = DeviceState();
     }
     cudaSetDevice(cur);
@@ -586,6 +637,7 @@ lf_status lf_attn_fwd_static(const void* q, const void* k, const void* v, void* 
     // never grows (allocates) it.  Prep zeroes what must start at zero.
     DeviceState view;
     view.init = true;
+    view.may_order = false;
     view.sm_count = ss->sm_count;
     view.status = reinterpret_cast<uint32_t*>(ss->scratch);
     view.ws = ss->scratch + 256;

@@ -86,6 +86,7 @@ struct BandTcParams {
     int dk_rows[kMaxDilKinds];   // rows per TMA box for that dilation
     int head_start[kMaxHeads + 1];  // item offset of each head inside one sample
     uint8_t head_dk[kMaxHeads];
+    const int32_t* item_order;  // work slot -> item (longest tiles first); null: slot = item
 };
 
 }  // namespace lf
