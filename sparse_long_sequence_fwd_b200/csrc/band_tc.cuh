@@ -539,7 +539,6 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
 
             if (!wait_warp(&bars[kBarSFull], g & 1u)) return;
             tc_fence_after();
-            if (!ensure_p_ready()) return;
             float lsum[4] = {0.f, 0.f, 0.f, 0.f};
             // one body for every chunk: a second copy (for a load in flight during the
             // previous chunk) costs more in instruction fetch than it hides
@@ -612,7 +611,10 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                         lsum[2] *= alpha;
                         lsum[3] *= alpha;
                     }
-                    if (c > 0 || blk > 0) rescale_held(tP, c, tO, blk > 0, alpha);
+                    if (c > 0 || blk > 0) {
+                        if (!ensure_p_ready()) return;
+                        rescale_held(tP, c, tO, blk > 0, alpha);
+                    }
                 }
                 const float nb2 = (m_ref == -INFINITY) ? 0.f : -m_ref;
                 uint32_t pk[16];
@@ -623,6 +625,8 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                     lsum[(j >> 1) & 3] += e0 + e1;
                     pk[j >> 1] = pack_bf16x2(e0, e1);
                 }
+                // the previous product is waited for only here, after chunk 0's work
+                if (c == 0 && !ensure_p_ready()) return;
                 tmem_st16(tP + 16u * c, pk);
             }
             l_row += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
