@@ -93,9 +93,13 @@ lf_status lf_attn_fwd(const void* q, const void* k, const void* v, void* out,
  *
  * q, k, v, out, global_idx and key_pad_mask are host pointers with the
  * layouts above (page-locked memory gives full copy bandwidth).  The call
- * copies the inputs into a library-owned device staging area on `stream`,
- * runs lf_attn_fwd, copies `out` back and synchronises `stream`, so `out`
- * is ready when it returns.
+ * copies the inputs into a library-owned device staging area, runs the
+ * forward and copies `out` back, ordered after the work already queued on
+ * `stream`, and returns when `out` is ready.  It works on up to 8 slices
+ * of (sample, group of heads): the inputs of a slice are copied on a
+ * library-owned copy-in stream, its kernels run on `stream`, and its output
+ * is copied back on a copy-out stream, so the copies of one slice overlap
+ * the kernels and copies of the others.
  */
 lf_status lf_attn_fwd_host(const void* q, const void* k, const void* v, void* out,
                            int B, int H, int T, int d, int r, const int32_t* dil,

@@ -41,6 +41,11 @@ struct DeviceState {
     // finish; null: everything runs in order on the caller's stream.
     cudaStream_t aux = nullptr;
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    // lf_attn_fwd_host: copy-in / copy-out streams and per-slice events, so the
+    // copies of one slice overlap the kernels of another
+    static constexpr int kMaxSlices = 8;
+    cudaStream_t cin = nullptr, cout = nullptr;
+    cudaEvent_t ev_in[kMaxSlices] = {}, ev_done[kMaxSlices] = {};
     // Band work items in longest-first order (device copy), for the shape in
     // order_key; rebuilt outside stream capture when the shape changes.
     bool may_order = true;  // false: never allocate for it (the allocation-free entry point)
@@ -139,8 +144,14 @@ lf_status device_state(DeviceState** out) {
         if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
             cudaStreamCreateWithPriority(&s.aux, cudaStreamNonBlocking, least) != cudaSuccess ||
             cudaEventCreateWithFlags(&s.ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&s.ev_join, cudaEventDisableTiming) != cudaSuccess)
+            cudaEventCreateWithFlags(&s.ev_join, cudaEventDisableTiming) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&s.cin, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&s.cout, cudaStreamNonBlocking) != cudaSuccess)
             return LF_ERR_CUDA;
+        for (int a = 0; a < DeviceState::kMaxSlices; ++a)
+            if (cudaEventCreateWithFlags(&s.ev_in[a], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&s.ev_done[a], cudaEventDisableTiming) != cudaSuccess)
+                return LF_ERR_CUDA;
         s.init = true;
     }
     *out = &s;
@@ -548,23 +559,64 @@ lf_status lf_attn_fwd_host(const void* q, const void* k, const void* v, void* ou
     const size_t total = o_p + align256(size_t(B) * T);
     if ((st = grow(&ds->io, &ds->io_bytes, total, s)) != LF_OK) return st;
     uint8_t* io = static_cast<uint8_t*>(ds->io);
-    if (cudaMemcpyAsync(io + o_q, q, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(io + o_k, k, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(io + o_v, v, nb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    // The copies stay ordered after the work already queued on `s`.
+    if (cudaEventRecord(ds->ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(ds->cin, ds->ev_fork, 0) != cudaSuccess)
         return LF_ERR_CUDA;
+    // Small inputs first (global lists and padding of every sample), on the copy-in stream.
     if (n_global > 0 &&
-        cudaMemcpyAsync(io + o_g, global_idx, sizeof(int32_t) * size_t(B) * n_global, cudaMemcpyHostToDevice, s) !=
-            cudaSuccess)
+        cudaMemcpyAsync(io + o_g, global_idx, sizeof(int32_t) * size_t(B) * n_global, cudaMemcpyHostToDevice,
+                        ds->cin) != cudaSuccess)
         return LF_ERR_CUDA;
-    if (key_pad_mask && cudaMemcpyAsync(io + o_p, key_pad_mask, size_t(B) * T, cudaMemcpyHostToDevice, s) !=
+    if (key_pad_mask && cudaMemcpyAsync(io + o_p, key_pad_mask, size_t(B) * T, cudaMemcpyHostToDevice, ds->cin) !=
                             cudaSuccess)
         return LF_ERR_CUDA;
-    st = launch_all(io + o_q, io + o_k, io + o_v, io + o_o, B, H, T, d, r, dil,
-                    n_global > 0 ? reinterpret_cast<const int32_t*>(io + o_g) : nullptr, n_global,
-                    key_pad_mask ? io + o_p : nullptr, scale, dtype, s, ds);
+    // Slices of (sample, group of heads), each an independent problem: its q, k, v go in
+    // on the copy-in stream, its kernels run on `s` once they have landed, and its
+    // output goes back on the copy-out stream, so the copies of one slice overlap the
+    // kernels and copies of the others.  The kernels of the slices share the workspace
+    // in stream order on `s`.
+    const int groups = std::max(1, std::min(H, (DeviceState::kMaxSlices + B - 1) / B));
+    const int hg = (H + groups - 1) / groups;
+    const int nslices = B * ((H + hg - 1) / hg);
+    const bool sliced = nslices > 1 && nslices <= DeviceState::kMaxSlices;
+    const int slice_h = sliced ? hg : H;
+    const size_t per_head = size_t(T) * d * es;
+    const bool saved_order = ds->may_order;
+    ds->may_order = !sliced;  // one tile order per call: the slices would keep rebuilding it
+    int a = 0;
+    for (int b = 0; b < (sliced ? B : 1) && st == LF_OK; ++b)
+        for (int h0 = 0; h0 < H && st == LF_OK; h0 += slice_h, ++a) {
+            const int nh = sliced ? std::min(slice_h, H - h0) : H;
+            const int bb = sliced ? 1 : B;
+            const size_t off = (size_t(b) * H + h0) * per_head, bytes = size_t(bb) * nh * per_head;
+            cudaEvent_t ev_in = ds->ev_in[a], ev_done = ds->ev_done[a];
+            if (cudaMemcpyAsync(io + o_q + off, static_cast<const uint8_t*>(q) + off, bytes, cudaMemcpyHostToDevice,
+                                ds->cin) != cudaSuccess ||
+                cudaMemcpyAsync(io + o_k + off, static_cast<const uint8_t*>(k) + off, bytes, cudaMemcpyHostToDevice,
+                                ds->cin) != cudaSuccess ||
+                cudaMemcpyAsync(io + o_v + off, static_cast<const uint8_t*>(v) + off, bytes, cudaMemcpyHostToDevice,
+                                ds->cin) != cudaSuccess ||
+                cudaEventRecord(ev_in, ds->cin) != cudaSuccess || cudaStreamWaitEvent(s, ev_in, 0) != cudaSuccess) {
+                st = LF_ERR_CUDA;
+                break;
+            }
+            const int32_t* gdev = n_global > 0 ? reinterpret_cast<const int32_t*>(io + o_g) + size_t(b) * n_global
+                                               : nullptr;
+            const uint8_t* pdev = key_pad_mask ? io + o_p + size_t(b) * T : nullptr;
+            st = launch_all(io + o_q + off, io + o_k + off, io + o_v + off, io + o_o + off, bb, nh, T, d, r,
+                            dil ? dil + h0 : nullptr, gdev, n_global, pdev, scale, dtype, s, ds);
+            if (st != LF_OK) break;
+            if (cudaEventRecord(ev_done, s) != cudaSuccess || cudaStreamWaitEvent(ds->cout, ev_done, 0) != cudaSuccess ||
+                cudaMemcpyAsync(static_cast<uint8_t*>(out) + off, io + o_o + off, bytes, cudaMemcpyDeviceToHost,
+                                ds->cout) != cudaSuccess)
+                st = LF_ERR_CUDA;
+        }
+    ds->may_order = saved_order;
+    // everything queued so far must finish before the staging area is reused or `out` is read
+    const bool synced = cudaStreamSynchronize(ds->cin) == cudaSuccess &&
+                        cudaStreamSynchronize(s) == cudaSuccess && cudaStreamSynchronize(ds->cout) == cudaSuccess;
     if (st != LF_OK) return st;
-    if (cudaMemcpyAsync(out, io + o_o, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return LF_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return LF_ERR_CUDA;
+    if (!synced) return LF_ERR_CUDA;
     return LF_OK;
 }
 
@@ -611,6 +663,12 @@ void lf_attn_release(void) {
         if (s.ev_fork) cudaEventDestroy(s.ev_fork);
         if (s.ev_join) cudaEventDestroy(s.ev_join);
         if (s.aux) cudaStreamDestroy(s.aux);
+        if (s.cin) cudaStreamDestroy(s.cin);
+        if (s.cout) cudaStreamDestroy(s.cout);
+        for (int a = 0; a < DeviceState::kMaxSlices; ++a) {
+            if (s.ev_in[a]) cudaEventDestroy(s.ev_in[a]);
+            if (s.ev_done[a]) cudaEventDestroy(s.ev_done[a]);
+        }
         s = DeviceState();
     }
     cudaSetDevice(cur);

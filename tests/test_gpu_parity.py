@@ -191,6 +191,21 @@ def test_host_entry_point_matches_device_entry_point():
     assert torch.equal(host, dev.cpu())
 
 
+def test_host_entry_point_slices_heads_with_their_dilations():
+    """The host entry point runs each head of this call as its own slice (its
+    own dilation and the sample's globals and padding): same output as the
+    device entry point, bit for bit."""
+    w = workloads.custom("host_dil", "bf16", 1, 6, 900, 64, 40, dil=[1, 1, 2, 2, 3, 3], globals_per_b=[[4, 800]],
+                         pad_from=[850], seed=43)
+    inp = workloads.make_inputs(w)
+    dev = parity.run_gpu(w, inp)
+    pinned = {k: (v.pin_memory() if isinstance(v, torch.Tensor) and k != "dil" else v) for k, v in inp.items()}
+    host = lf_attn.fwd_host(pinned["q"], pinned["k"], pinned["v"], w.r, dil=inp["dil"],
+                            global_idx=pinned["global_idx"], key_pad_mask=pinned["key_pad_mask"],
+                            scale=w.softmax_scale)
+    assert torch.equal(host, dev.cpu())
+
+
 def test_argument_errors_on_gpu_do_not_launch():
     q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(lf_attn.LfAttnError) as e:
