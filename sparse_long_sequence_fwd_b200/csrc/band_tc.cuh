@@ -16,17 +16,19 @@
 // Per key block:   S = Q K^T        tcgen05.mma, M=128, N=128 (or the global
 //                                   count rounded to 16), K=64, operands in
 //                                   shared memory -> S in TMEM (fp32)
-//                  online softmax   one thread per query row (TMEM lane), all
-//                                   128 columns of the block in registers;
+//                  online softmax   one thread per query row (TMEM lane),
+//                                   the block read in four 32-column chunks;
 //                                   running max, exponent base and row sum
 //                                   in fp32, log2 domain
 //                  O += P V         P (bf16) written back to TMEM by the
 //                                   softmax threads and read from there as
 //                                   the A operand; V from shared memory;
 //                                   M=128, N=64, K=128
-// The exponent base only moves (O and the row sum rescaled in place) when a
-// block's max exceeds it by more than 2^8; otherwise p = 2^(s - base) stays
-// below 256, which fp32 accumulation and bf16 P absorb.
+// The exponent base only moves (O and the row sum rescaled in place) between
+// blocks, when the max seen exceeds it by more than 2^8; otherwise
+// p = 2^(s - base) stays below 256, which fp32 accumulation and bf16 P absorb
+// (a jump of more than 2^64 inside a block is handled at once, see the
+// softmax role).
 // The mask view of the note ("Mask View": A = QK^T/sqrt(d) + M, M = -inf off
 // the pattern) is applied inline: band limits and sequence ends as a per-row
 // column interval, padded keys from the key padding mask, the global-key
@@ -343,9 +345,9 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
 
 // ------------------------------------------------------------ softmax role
 // Thread x owns query row x of the tile (TMEM lane x) and walks each S block
-// in four chunks of 32 columns: the TMEM load of chunk c + 1 is in flight
-// while chunk c is exponentiated and its P (16 columns of bf16 pairs) is
-// stored, so only two chunks of S are ever held in registers.
+// in four chunks of 32 columns, one loop body for all of them: TMEM load,
+// mask, max, exponentials, P (16 columns of bf16 pairs) back to TMEM, so
+// only one chunk of S is held in registers.
 //
 // Exponent base.  p = 2^(s*sl2 - base) with base = m_ref.  The base moves
 // between blocks, to the largest scaled score seen so far, once that exceeds
