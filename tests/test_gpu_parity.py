@@ -5,10 +5,12 @@
   span several 128-row tiles, a ragged tail, several residue classes,
   padding and more than one 128-wide block of global keys: every element;
 * the four full-size bf16 workloads in the launch configuration the bench
-  times: the base workload in full, the others on sampled rows;
+  times, every element against the full oracle (plus a quick sampled-row
+  check of the same three larger ones);
 * edge cases: T < w, r = 0, no globals, global at T-1, padded globals,
   an all-padded sample, T mod dil != 0, duplicates, out-of-range entries.
-bf16 bar: max-abs <= 2e-2 and relative RMS <= 5e-3 over the compared rows.
+bf16 bar: max-abs <= 2e-2 and relative RMS <= 5e-3 over the whole tensor
+(over the compared rows for the sampled-row check).
 """
 import numpy as np
 import pytest
@@ -65,6 +67,14 @@ def test_base_workload_every_element():
 
 
 @pytest.mark.parametrize("w", [workloads.QA, workloads.DILATED, workloads.LARGE], ids=lambda w: w.name)
+def test_full_size_workloads_every_element(w):
+    """QA (two samples, 64 globals, padding), dilated (dilation 1 and 2) and
+    large (T = 16384, 32 random globals): every element of the output against
+    the full oracle, max-abs and relative RMS over the whole tensor."""
+    _full_case(w)
+
+
+@pytest.mark.parametrize("w", [workloads.QA, workloads.DILATED, workloads.LARGE], ids=lambda w: w.name)
 def test_full_size_workloads_sampled_rows(w):
     inp = workloads.make_inputs(w)
     got = parity.run_gpu(w, inp)
@@ -97,6 +107,10 @@ EDGES = [
     workloads.custom("scale_big", "bf16", 1, 2, 900, 64, 256, globals_per_b=[[3, 700]], scale=2.0, seed=35),
     workloads.custom("scale_big_f32", "f32", 1, 2, 300, 32, 40, globals_per_b=[[3]], scale=2.0, seed=36),
     workloads.custom("scale_negative", "bf16", 1, 2, 400, 64, 60, globals_per_b=[[0]], scale=-0.3, seed=37),
+    # scale 0: every kept key gets the same weight, so each row is the mean of V over N(i)
+    workloads.custom("scale_zero", "bf16", 1, 2, 400, 64, 60, dil=[1, 2], globals_per_b=[[0, 333]],
+                     pad_from=[390], scale=0.0, seed=44),
+    workloads.custom("scale_zero_f32", "f32", 1, 2, 120, 16, 9, globals_per_b=[[5]], scale=0.0, seed=45),
 ]
 
 
