@@ -146,6 +146,36 @@ uint64_t lf_attn_workspace_bytes(int B, int H, int T, int d, int n_global, lf_dt
 int lf_attn_last_launch_count(void);
 
 /*
+ * lf_attn_test_hooks -- test hook for the device-side failure path (no
+ * counterpart in the pages).  wait_ns sets the limit of every pipeline wait
+ * of the bf16 band kernel in later calls (0 restores the default, 1 s);
+ * flags bit 0 makes the band kernel's producers stop before their first
+ * load, so the other roles' waits run out, the kernel ends early with
+ * status bit 1 set (lf_attn_device_status reports LF_ERR_DEVICE_CHECK) and
+ * that call's output is not written.  Nothing faults or hangs; a later call
+ * with lf_attn_test_hooks(0, 0) computes normally.  Process-wide setting.
+ */
+void lf_attn_test_hooks(uint32_t flags, uint64_t wait_ns);
+
+/*
+ * lf_attn_band_plan -- diagnostic: how the bf16 band kernel splits its work
+ * for these sizes over at most max_ctas CTAs, computed on the host by the
+ * same code the kernel's producer runs (no device is touched).  The tiles'
+ * key blocks form one sequence (per sample, heads; per head, residue
+ * classes of the dilation; per class, 128-query tiles; per tile, its band
+ * blocks then its global-key blocks), and CTA s takes an equal contiguous
+ * share of it, cutting tiles into pieces where needed.
+ *   pieces: host array of capacity x 10 int32 (may be NULL); piece k gets
+ *     {cta, tile, first block, end block, blocks of the tile, first CTA of
+ *      the tile, last CTA of the tile, partial-state slot, b*H + h,
+ *      class * 65536 + tile within the class}.
+ * Returns the number of pieces (which may exceed capacity), or -1 for
+ * invalid or unsupported sizes.
+ */
+int lf_attn_band_plan(int B, int H, int T, int r, const int32_t* dil, int n_global, int max_ctas,
+                      int32_t* pieces, int capacity);
+
+/*
  * lf_attn_fwd_static -- lf_attn_fwd for callers that cannot allocate device
  * memory (the pages describe no counterpart; this is a deployment variant).
  *

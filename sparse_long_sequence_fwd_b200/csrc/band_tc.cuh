@@ -1,39 +1,49 @@
 // band_tc.cuh -- K1: fused band kernel for bf16, d = 64, on the 5th-generation
 // tensor cores (tcgen05) with TMA staging and TMEM accumulators.
 //
-// Work item = 128 consecutive queries of one residue class c of one (b, h):
-// rows i = c + dil*(q0 + x), x in [0, 128).  Inside a class the dilated
-// window {i + dil*t : |t| <= r} ("Longformer" wiki, section 2.2.3; the
-// "Longformer" note, section "Sliding-Window Attention") is a dense window
-// of radius r over the class's own positions, so the item needs the key
-// rows of its diagonal band only: decimated keys [q0 - r, q0 + 127 + r],
-// fetched in blocks of 128 with TMA boxes whose row traversal stride is dil.
-// After the band blocks come ceil(n_gk / 128) blocks of packed global keys
-// (built by the prep kernel), masked where a global key already lies in the
-// row's window so each key counts once ("Global Attention": N(i) = N_local(i)
-// U G).
+// Tile = 128 consecutive queries of one residue class c of one (b, h): rows
+// i = c + dil*(q0 + x), x in [0, 128).  Inside a class the dilated window
+// {i + dil*t : |t| <= r} ("Longformer" wiki, section 2.2.3; the "Longformer"
+// note, section "Sliding-Window Attention") is a dense window of radius r
+// over the class's own positions, so a tile needs the key rows of its
+// diagonal band only: decimated keys [q0 - r, q0 + 127 + r], fetched in
+// blocks of 64 with TMA boxes whose row traversal stride is dil.  After the
+// band blocks come ngb blocks of packed global keys (built by the prep
+// kernel), masked where a global key already lies in the row's window so
+// each key counts once ("Global Attention": N(i) = N_local(i) U G).
 //
-// Per key block:   S = Q K^T        tcgen05.mma, M=128, N=128 (or the global
+// Per key block:   S = Q K^T        tcgen05.mma, M=128, N=64 (or the global
 //                                   count rounded to 16), K=64, operands in
 //                                   shared memory -> S in TMEM (fp32)
-//                  online softmax   one thread per query row (TMEM lane),
-//                                   the block read in four 32-column chunks;
-//                                   running max, exponent base and row sum
-//                                   in fp32, log2 domain
-//                  O += P V         P (bf16) written back to TMEM by the
-//                                   softmax threads and read from there as
-//                                   the A operand; V from shared memory;
-//                                   M=128, N=64, K=128
-// The exponent base only moves (O and the row sum rescaled in place) between
-// blocks, when the max seen exceeds it by more than 2^8; otherwise
-// p = 2^(s - base) stays below 256, which fp32 accumulation and bf16 P absorb
-// (a jump of more than 2^64 inside a block is handled at once, see the
-// softmax role).
+//                  online softmax   one thread per query row (TMEM lane): the
+//                                   row's 64 scores in registers, masked,
+//                                   block max, exponent base, exp2, row sum
+//                  O += P V         P (bf16) written over the S block it came
+//                                   from and read from TMEM as the A operand;
+//                                   V from shared memory; M=128, N=64, K=64
+// S lives in a ring of three TMEM buffers, so the products of the next blocks
+// are ready while the softmax threads work on this one: in steady state the
+// softmax threads wait for nothing but S.  The exponent base moves (O and the
+// row sum rescaled in place) only when a block's max exceeds it by more than
+// 2^8; otherwise p = 2^(s - base) stays below 256, which fp32 accumulation
+// and bf16 P absorb.
 // The mask view of the note ("Mask View": A = QK^T/sqrt(d) + M, M = -inf off
 // the pattern) is applied inline: band limits and sequence ends as a per-row
 // column interval, padded keys from the key padding mask, the global-key
-// dedup test per column.  Blocks that lie inside every row's window need no
-// test at all.  Nothing of size T x T is built.
+// dedup test per column.  Blocks inside every row's window need no test, and
+// 32-column chunks that no row of a warp keeps skip their exponentials.
+// Nothing of size T x T is built.
+//
+// Work split ("stream-K").  The tiles' key blocks, in the order (b, h, c,
+// tile, block), form one sequence; CTA s takes the contiguous range
+// [s*N/G, (s+1)*N/G) of it, so every CTA gets the same number of blocks
+// whatever the tile count.  A range boundary that cuts a tile leaves pieces
+// of it in neighbouring CTAs; each piece ends with its partial softmax state
+// (m, l, O) per row.  Per 32-row quarter, each piece takes a ticket (atomic)
+// as it starts its last block; the last to arrive merges the partial states,
+// which the others write to the workspace without waiting for anything, in
+// CTA order (so the result does not depend on who arrives last), and stores
+// the rows.  A piece only ever waits for pieces that have already arrived.
 //
 // Two CTAs share an SM (96 KB of shared memory and 256 TMEM columns each):
 // while one CTA's softmax warps wait on a barrier or a TMEM load, the
@@ -47,83 +57,177 @@
 
 namespace lf {
 
-constexpr int kBM = 128;
-constexpr int kBN = 128;
+constexpr int kBM = 128;  // queries per tile
+constexpr int kBN = 64;   // keys per block
 constexpr int kHD = 64;
-constexpr int kStages = 2;                 // Q, K and V rings
-constexpr int kTileBytes = kBM * kHD * 2;  // 16 KB: 128 rows x 128 bytes
+constexpr int kQStages = 2;
+constexpr int kKVStages = 4;
+constexpr int kSBufs = 3;                // S / P buffers in TMEM
+constexpr int kQBytes = kBM * kHD * 2;   // 16 KB: 128 rows x 128 bytes
+constexpr int kKVBytes = kBN * kHD * 2;  // 8 KB
 constexpr int kBandThreads = 192;
 constexpr int kBandCtasPerSm = 2;
-constexpr int kSoftmaxWarp0 = 2;  // warps 2..5
 constexpr int kSoftmaxWarps = 4;
 constexpr float kRescaleLog2 = 8.f;  // move the exponent base only past 2^8
 
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kStages * kTileBytes;
-constexpr int kOffV = kOffK + kStages * kTileBytes;
-constexpr int kOffBar = kOffV + kStages * kTileBytes;
+constexpr int kOffK = kOffQ + kQStages * kQBytes;
+constexpr int kOffV = kOffK + kKVStages * kKVBytes;
+constexpr int kOffBar = kOffV + kKVStages * kKVBytes;
 // barrier slots
-constexpr int kBarQFull = 0, kBarQEmpty = kBarQFull + kStages, kBarKFull = kBarQEmpty + kStages,
-              kBarKEmpty = kBarKFull + kStages, kBarVFull = kBarKEmpty + kStages, kBarVEmpty = kBarVFull + kStages,
-              kBarSFull = kBarVEmpty + kStages, kBarSFree = kBarSFull + 1, kBarPFull = kBarSFree + 1,
-              kBarOFull = kBarPFull + 1, kBarDrain = kBarOFull + 1, kNumBars = kBarDrain + 1;
-// Tile descriptors (BandTile), one per Q slot: written by the producer before
-// it arrives on the slot's Q-full barrier, read by the MMA and softmax roles
-// after waiting on it, so only the producer decodes work items.
+constexpr int kBarQFull = 0, kBarQEmpty = kBarQFull + kQStages, kBarKFull = kBarQEmpty + kQStages,
+              kBarKEmpty = kBarKFull + kKVStages, kBarVFull = kBarKEmpty + kKVStages,
+              kBarVEmpty = kBarVFull + kKVStages, kBarSFull = kBarVEmpty + kKVStages, kBarPFull = kBarSFull + kSBufs,
+              kBarBufFree = kBarPFull + kSBufs, kBarOFull = kBarBufFree + kSBufs, kBarDrain = kBarOFull + 2,
+              kNumBars = kBarDrain + 1;
+// Piece descriptors (BandPiece), one per Q slot: written by the producer
+// before it arrives on the slot's Q-full barrier, read by the MMA and softmax
+// roles after waiting on it, so only the producer walks the work sequence.
+// A slot (Q tile and descriptor) is free again once the piece's last
+// product has been issued and its rows have been written.
 constexpr int kOffDesc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
-constexpr int kDescBytes = 64;
-constexpr int kOffMisc = kOffDesc + kStages * kDescBytes;
+constexpr int kDescBytes = 128;
+constexpr int kOffMisc = kOffDesc + kQStages * kDescBytes;
 constexpr int kMiscBytes = 16;
 constexpr int kBandSmem = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 static_assert(kBandCtasPerSm * (kBandSmem + 1024) <= 233472, "shared memory budget for two CTAs per SM");
 
-// TMEM columns (256 per CTA): S (fp32, 128 wide) at 0, P (bf16 pairs, 64
-// wide) at 128, O (fp32, 64 wide) at 192.
+// TMEM columns (256 per CTA): three S buffers of 64 fp32 columns at 0, 64,
+// 128 (P, bf16 pairs, over the first 32 columns of its own buffer), O (fp32,
+// 64 wide) at 192.
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
+constexpr uint32_t kColO = 192;
 
-struct BandTile {
+// Partial state of one piece (128 rows): O as [16][128][4] fp32 (four
+// columns of every row per 16-byte group, so a warp's stores and loads are
+// contiguous), then m[128] and l[128].
+constexpr int kPartFloats = kBM * kHD + 2 * kBM;
+
+// One piece: blocks [blk_lo, blk_hi) of one tile's nbb band blocks and ngb
+// global blocks.
+struct BandPiece {
     int b, bh, c, dil, dk, R;
-    int Tc, q0, kbase, kb_lo, nbb, ngk, ngb;
+    int Tc, q0, kbase, kb_lo, nbb, ngb;
+    int blk_lo, blk_hi;
+    int tile;          // tile index (its merge tickets)
+    int s0, s1;        // the CTAs whose ranges hold the tile's blocks
+    int last;          // 1: the last piece this CTA processes
+    int tstart;        // position of the tile's first block in the sequence
 };
-static_assert(sizeof(BandTile) <= kDescBytes, "tile descriptor slot");
+static_assert(sizeof(BandPiece) <= kDescBytes, "piece descriptor slot");
 
-// Out of line: every role walks the same tiles, and one copy of this code
-// (integer divisions included) keeps the kernel small.
-__device__ __noinline__ BandTile band_decode(const BandTcParams& p, int item) {
-    BandTile t;
-    t.b = item / p.items_per_b;
-    int rem = item - t.b * p.items_per_b;
-    int h = 0;
-    while (p.head_start[h + 1] <= rem) ++h;
-    rem -= p.head_start[h];
-    t.bh = t.b * p.H + h;
-    t.dk = p.head_dk[h];
-    t.dil = p.dk_dil[t.dk];
-    t.R = p.dk_rows[t.dk];
-    int c = 0, Tc = 0;
-    for (c = 0; c < t.dil; ++c) {
-        Tc = (p.T - c + t.dil - 1) / t.dil;
-        const int nt = (Tc + kBM - 1) / kBM;
-        if (rem < nt) break;
-        rem -= nt;
-    }
-    t.c = c;
-    t.Tc = Tc;
-    t.q0 = rem * kBM;
-    t.kbase = t.q0 - p.r;
-    const int lo = max(0, t.kbase);
-    const int hi = min(Tc - 1, t.q0 + kBM - 1 + p.r);
-    t.kb_lo = (lo - t.kbase) / kBN;
-    t.nbb = (hi - t.kbase) / kBN + 1 - t.kb_lo;
-    t.ngk = p.n_gk[t.b];
-    t.ngb = (t.ngk + kBN - 1) / kBN;
-    return t;
+// Band blocks of tile t of a class with Tc decimated rows: the decimated keys
+// [q0 - r, q0 + 127 + r] clipped to [0, Tc), in kBN-key blocks counted from
+// kbase = q0 - r.
+__host__ __device__ __forceinline__ void tile_band(int Tc, int r, int t, int& kbase, int& kb_lo, int& nbb) {
+    const int q0 = t * kBM;
+    kbase = q0 - r;
+    const int lo = kbase > 0 ? kbase : 0;
+    const int hi = (q0 + kBM - 1 + r) < (Tc - 1) ? (q0 + kBM - 1 + r) : (Tc - 1);
+    kb_lo = (lo - kbase) / kBN;
+    nbb = (hi - kbase) / kBN + 1 - kb_lo;
 }
 
-// Columns of global block gb that the MMA computes (multiple of 16).
+// First block of CTA s's range, floor(s * N / G), from N = q * G + rm
+// (32-bit arithmetic: N < 2^31, G <= 296).
+__host__ __device__ __forceinline__ int range_start(const BandTcParams& p, int s) {
+    return p.blk_q * s + (p.blk_rm * s) / p.grid_ctas;
+}
+// The CTA whose range holds block x (every range has q or q + 1 blocks).
+__host__ __device__ __forceinline__ int cta_of(const BandTcParams& p, int x) {
+    int s = static_cast<int>(static_cast<double>(x) * p.grid_ctas / p.n_blocks);
+    while (s + 1 < p.grid_ctas && range_start(p, s + 1) <= x) ++s;
+    while (s > 0 && range_start(p, s) > x) --s;
+    return s;
+}
+
+// Walks the tiles in sequence order.
+struct TileWalker {
+    int b, h, c, t, tile;
+    int dk, dil, Tc, nt;
+    int kbase, kb_lo, nbb;
+    int start;  // position of the tile's first block
+
+    __host__ __device__ void set_class(const BandTcParams& p) {
+        dk = p.head_dk[h];
+        dil = p.dk_dil[dk];
+        Tc = (p.T - c + dil - 1) / dil;
+        nt = (Tc + kBM - 1) / kBM;
+    }
+    __host__ __device__ void shape(const BandTcParams& p) { tile_band(Tc, p.r, t, kbase, kb_lo, nbb); }
+    __host__ __device__ int nb(const BandTcParams& p) const { return nbb + p.ngb; }
+
+    // The tile that holds block x of the sequence.
+    __host__ __device__ void locate(const BandTcParams& p, int x) {
+        b = x / p.blocks_per_b;
+        int rem = x - b * p.blocks_per_b;
+        h = 0;
+        while (h + 1 < p.H && p.head_blk[h + 1] <= rem) ++h;
+        rem -= p.head_blk[h];
+        c = 0;
+        dk = p.head_dk[h];
+        while (c + 1 < p.dk_dil[dk] && p.dk_class_blk[dk][c + 1] <= rem) ++c;
+        rem -= p.dk_class_blk[dk][c];
+        set_class(p);
+        tile = b * p.tiles_per_b + p.head_tile[h] + p.dk_class_tile[dk][c];
+        start = x - rem;
+        // interior tiles (whole band inside [0, Tc)) all have the same block count
+        const int t_a = (p.r + kBM - 1) / kBM;
+        const int t_b = Tc - kBM - p.r >= 0 ? (Tc - kBM - p.r) / kBM + 1 : 0;
+        t = 0;
+        for (;;) {
+            shape(p);
+            const int n = nb(p);
+            if (t == t_a && t_b > t_a) {
+                const int span = (t_b - t_a) * n;
+                if (rem >= span) {
+                    rem -= span;
+                    start += span;
+                    tile += t_b - t_a;
+                    t = t_b;
+                    continue;
+                }
+                const int k = rem / n;
+                rem -= k * n;
+                start += k * n;
+                tile += k;
+                t += k;
+                shape(p);
+                break;
+            }
+            if (rem < n) break;
+            rem -= n;
+            start += n;
+            ++tile;
+            ++t;
+        }
+    }
+    // The next tile (residue classes with no rows, T < dil, are skipped).
+    __host__ __device__ void next(const BandTcParams& p) {
+        start += nb(p);
+        ++tile;
+        if (++t >= nt) {
+            t = 0;
+            do {
+                if (++c >= dil) {
+                    c = 0;
+                    if (++h == p.H) {
+                        h = 0;
+                        ++b;
+                    }
+                }
+                set_class(p);
+            } while (nt == 0);
+        }
+        shape(p);
+    }
+};
+
+// Columns of global block gb that the MMA computes (a multiple of 16, at
+// least 16 even where the block holds no key of this sample).
 __device__ __forceinline__ int global_block_cols(int ngk, int gb) {
-    const int rem = min(kBN, ngk - gb * kBN);
+    int rem = ngk - gb * kBN;
+    rem = rem < 16 ? 16 : (rem > kBN ? kBN : rem);
     return (rem + 15) & ~15;
 }
 
@@ -147,282 +251,416 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
-
-// Work item of a slot: the CTA with blockIdx b takes slots b, b + grid, ...;
-// the host may order the items so the longest tiles come first.
-__device__ __forceinline__ int slot_item(const BandTcParams& p, int slot) {
-    return p.item_order ? __ldg(p.item_order + slot) : slot;
+// Largest / smallest of 32 consecutive scores (four independent chains).
+__device__ __forceinline__ float max32(const uint32_t* v) {
+    float m[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m[u] = fmaxf(__uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]));
+#pragma unroll
+    for (int j = 8; j < 32; j += 8)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) m[u] = fmax3(m[u], __uint_as_float(v[j + 2 * u]), __uint_as_float(v[j + 2 * u + 1]));
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+__device__ __forceinline__ float min32(const uint32_t* v) {
+    float m[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m[u] = fminf(__uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]));
+#pragma unroll
+    for (int j = 8; j < 32; j += 8)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) m[u] = fmin3(m[u], __uint_as_float(v[j + 2 * u]), __uint_as_float(v[j + 2 * u + 1]));
+    return fminf(fminf(m[0], m[1]), fminf(m[2], m[3]));
 }
 
-// Walks the (slot, block) sequence of this CTA in the order every role uses.
-struct BlockCursor {
-    int item, blk, nb;
-    BandTile t;
-    __device__ __forceinline__ void start(const BandTcParams& p) {
-        item = blockIdx.x;
-        blk = 0;
-        if (item < p.n_items) {
-            t = band_decode(p, slot_item(p, item));
-            nb = t.nbb + t.ngb;
-        } else {
-            nb = 0;
-        }
-    }
-    __device__ __forceinline__ bool valid(const BandTcParams& p) const { return item < p.n_items; }
-    __device__ __forceinline__ void next(const BandTcParams& p) {
-        if (++blk < nb) return;
-        blk = 0;
-        item += gridDim.x;
-        if (item < p.n_items) {
-            t = band_decode(p, slot_item(p, item));
-            nb = t.nbb + t.ngb;
-        }
-    }
-};
-
 // ------------------------------------------------------------- TMA producer
-// K runs one block ahead of V: K(g + 1) is needed as soon as the softmax has
-// read S(g), V(g) only once P(g) is written.
+// Walks this CTA's range once: for each piece it publishes the descriptor and
+// loads the tile's Q, then the K and V blocks; K runs one block ahead of V
+// (K(g + 1) is needed for the next product, V(g) only once P(g) is written).
+// Processing order: when the range ends inside a tile (its head; the rest of
+// that tile is the first piece of the next CTA), that piece goes first, then
+// the range from its start.  Both pieces of every split tile are then done
+// early in their CTAs, so the merges that join them overlap other work
+// instead of ending the kernel.
+// Only the global-key blocks read the prep kernel's output (packed keys), so
+// the wait for prep comes just before the first of them: the band blocks of
+// the first tile overlap prep.
 __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                               volatile int* abort_flag) {
-    BlockCursor kc, vc;
-    kc.start(p);
-    vc.start(p);
+    const int s = blockIdx.x;
+    const int x0 = range_start(p, s);
+    const int x1 = range_start(p, s + 1);
+    TileWalker w;
+    w.locate(p, x0);
+    TileWalker wz = w;  // the tile that holds the range's last block: a few tiles on at most
+    while (wz.start + wz.nb(p) < x1) wz.next(p);
+    if (p.test_stall) return;  // test hook: nothing is published, so the other roles' waits run out
+    const bool front = wz.tile != w.tile && wz.start + wz.nb(p) > x1;  // the split last tile goes first
+    const int x_main_end = front ? wz.start : x1;
+    bool prep_done = false;
+
     uint32_t gk = 0, gv = 0, qt = 0;
-    auto issue_k = [&]() -> bool {
-        const BandTile& t = kc.t;
-        if (kc.blk == 0) {
+    auto issue_kv = [&](const BandPiece& d, int blk, bool is_v, uint32_t g) -> bool {
+        const uint32_t st = g % kKVStages;
+        const uint32_t ph = (g / kKVStages) & 1u;
+        uint64_t* empty = &bars[(is_v ? kBarVEmpty : kBarKEmpty) + st];
+        uint64_t* full = &bars[(is_v ? kBarVFull : kBarKFull) + st];
+        if (!mbar_wait(empty, ph ^ 1u, abort_flag, p.wait_ns)) return false;
+        uint8_t* dst = smem + (is_v ? kOffV : kOffK) + st * kKVBytes;
+        if (blk < d.nbb) {
+            mbar_arrive_expect_tx(full, kKVBytes);
+            const int j0 = d.kbase + kBN * (d.kb_lo + blk);
+            const CUtensorMap* tm = is_v ? &p.tm_v[d.dk] : &p.tm_k[d.dk];
+            for (int u = 0; u < kBN; u += d.R)
+                tma_load_3d(dst + u * 128, tm, full, 0, d.c + d.dil * (j0 + u), d.bh);
+        } else {
+            if (!prep_done) {  // packed global keys from here on
+                grid_dep_wait();
+                prep_done = true;
+            }
+            mbar_arrive_expect_tx(full, kKVBytes);
+            tma_load_3d(dst, is_v ? &p.tm_vg : &p.tm_kg, full, 0, (blk - d.nbb) * kBN, d.bh);
+        }
+        return true;
+    };
+
+    // current position: block x of tile cw, inside the segment that ends at x_stop
+    bool in_front = front;
+    TileWalker* cw = in_front ? &wz : &w;
+    int x = in_front ? wz.start : x0;
+    int x_stop = in_front ? x1 : x_main_end;
+    bool piece_start = true;
+    bool have_prev = false;
+    int prev_slot = 0, prev_blk = 0;
+    bool ok = true;
+    while (ok) {
+        const bool have_cur = x < x_stop;
+        int cur_slot = 0, cur_blk = 0;
+        if (have_cur) {
+            const int tend = cw->start + cw->nb(p);
+            const int blk = x - cw->start;
             const uint32_t qs = qt & 1u;
-            if (!mbar_wait(&bars[kBarQEmpty + qs], ((qt >> 1) & 1u) ^ 1u, abort_flag)) return false;
-            *reinterpret_cast<BandTile*>(smem + kOffDesc + qs * kDescBytes) = t;  // released by the arrive
-            mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes);
-            uint8_t* dQ = smem + kOffQ + qs * kTileBytes;
-            for (int u = 0; u < kBM; u += t.R)
-                tma_load_3d(dQ + u * 128, &p.tm_q[t.dk], &bars[kBarQFull + qs], 0, t.c + t.dil * (t.q0 + u), t.bh);
-            ++qt;
-        }
-        const uint32_t s = gk & 1u;
-        if (!mbar_wait(&bars[kBarKEmpty + s], ((gk >> 1) & 1u) ^ 1u, abort_flag)) return false;
-        mbar_arrive_expect_tx(&bars[kBarKFull + s], kTileBytes);
-        uint8_t* dK = smem + kOffK + s * kTileBytes;
-        if (kc.blk < t.nbb) {
-            const int j0 = t.kbase + kBN * (t.kb_lo + kc.blk);
-            for (int u = 0; u < kBN; u += t.R)
-                tma_load_3d(dK + u * 128, &p.tm_k[t.dk], &bars[kBarKFull + s], 0, t.c + t.dil * (j0 + u), t.bh);
-        } else {
-            tma_load_3d(dK, &p.tm_kg, &bars[kBarKFull + s], 0, (kc.blk - t.nbb) * kBN, t.bh);
-        }
-        ++gk;
-        return true;
-    };
-    auto issue_v = [&]() -> bool {
-        const BandTile& t = vc.t;
-        const uint32_t s = gv & 1u;
-        if (!mbar_wait(&bars[kBarVEmpty + s], ((gv >> 1) & 1u) ^ 1u, abort_flag)) return false;
-        mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes);
-        uint8_t* dV = smem + kOffV + s * kTileBytes;
-        if (vc.blk < t.nbb) {
-            const int j0 = t.kbase + kBN * (t.kb_lo + vc.blk);
-            for (int u = 0; u < kBN; u += t.R)
-                tma_load_3d(dV + u * 128, &p.tm_v[t.dk], &bars[kBarVFull + s], 0, t.c + t.dil * (j0 + u), t.bh);
-        } else {
-            tma_load_3d(dV, &p.tm_vg, &bars[kBarVFull + s], 0, (vc.blk - t.nbb) * kBN, t.bh);
-        }
-        ++gv;
-        return true;
-    };
-    bool first = true;
-    while (vc.valid(p)) {  // K(0); then K(g + 1), V(g) for g = 0, 1, ...
-        if (kc.valid(p)) {
-            if (!issue_k()) break;
-            kc.next(p);
-            if (first) {
-                first = false;
-                continue;
+            if (piece_start) {  // a new piece: descriptor and Q
+                piece_start = false;
+                if (!mbar_wait(&bars[kBarQEmpty + qs], ((qt >> 1) & 1u) ^ 1u, abort_flag, p.wait_ns)) break;
+                BandPiece d;
+                d.b = cw->b;
+                d.bh = cw->b * p.H + cw->h;
+                d.c = cw->c;
+                d.dil = cw->dil;
+                d.dk = cw->dk;
+                d.R = p.dk_rows[cw->dk];
+                d.Tc = cw->Tc;
+                d.q0 = cw->t * kBM;
+                d.kbase = cw->kbase;
+                d.kb_lo = cw->kb_lo;
+                d.nbb = cw->nbb;
+                d.ngb = p.ngb;
+                d.blk_lo = blk;
+                const int pend = tend < x_stop ? tend : x_stop;
+                d.blk_hi = pend - cw->start;
+                d.tile = cw->tile;
+                // the CTAs whose ranges hold the tile's blocks, found from this one
+                int s0 = s, s1 = s;
+                while (s0 > 0 && range_start(p, s0) > cw->start) --s0;
+                while (s1 + 1 < p.grid_ctas && range_start(p, s1 + 1) <= tend - 1) ++s1;
+                d.s0 = s0;
+                d.s1 = s1;
+                d.last = (!in_front && pend == x_main_end) ? 1 : 0;
+                d.tstart = cw->start;
+                *reinterpret_cast<BandPiece*>(smem + kOffDesc + qs * kDescBytes) = d;  // released by the arrive
+                mbar_arrive_expect_tx(&bars[kBarQFull + qs], kQBytes);
+                uint8_t* dQ = smem + kOffQ + qs * kQBytes;
+                for (int u = 0; u < kBM; u += d.R)
+                    tma_load_3d(dQ + u * 128, &p.tm_q[d.dk], &bars[kBarQFull + qs], 0, d.c + d.dil * (d.q0 + u), d.bh);
+                ++qt;
+            }
+            cur_slot = (qt - 1) & 1u;
+            cur_blk = blk;
+            const BandPiece& d = *reinterpret_cast<const BandPiece*>(smem + kOffDesc + cur_slot * kDescBytes);
+            if (!issue_kv(d, blk, false, gk)) break;
+            ++gk;
+            ++x;
+            if (x == x_stop || x == tend) {  // the piece ends here
+                piece_start = true;
+                if (x == x_stop && in_front) {  // on to the range from its start
+                    in_front = false;
+                    cw = &w;
+                    x = x0;
+                    x_stop = x_main_end;
+                } else if (x < x_stop) {
+                    cw->next(p);
+                }
             }
         }
-        if (!issue_v()) break;
-        vc.next(p);
+        if (have_prev) {
+            const BandPiece& d = *reinterpret_cast<const BandPiece*>(smem + kOffDesc + prev_slot * kDescBytes);
+            if (!issue_kv(d, prev_blk, true, gv)) break;
+            ++gv;
+        }
+        have_prev = have_cur;
+        prev_slot = cur_slot;
+        prev_blk = cur_blk;
+        ok = have_cur || have_prev;
     }
     if (*abort_flag) {  // let issued copies land before the CTA can exit
-        for (uint32_t s = 0; s < kStages; ++s) {
-            if (gk > s) (void)mbar_wait_drain(&bars[kBarKFull + s], ((gk - 1 - s) >> 1) & 1u);
-            if (gv > s) (void)mbar_wait_drain(&bars[kBarVFull + s], ((gv - 1 - s) >> 1) & 1u);
-            if (qt > s) (void)mbar_wait_drain(&bars[kBarQFull + s], ((qt - 1 - s) >> 1) & 1u);
+        for (uint32_t k = 0; k < kKVStages; ++k) {
+            if (gk > k) (void)mbar_wait_drain(&bars[kBarKFull + (gk - 1 - k) % kKVStages], ((gk - 1 - k) / kKVStages) & 1u);
+            if (gv > k) (void)mbar_wait_drain(&bars[kBarVFull + (gv - 1 - k) % kKVStages], ((gv - 1 - k) / kKVStages) & 1u);
         }
+        for (uint32_t k = 0; k < kQStages; ++k)
+            if (qt > k) (void)mbar_wait_drain(&bars[kBarQFull + ((qt - 1 - k) & 1u)], ((qt - 1 - k) >> 1) & 1u);
     }
 }
 
 // --------------------------------------------------------------- MMA issuer
-// S(g) = Q K(g)^T as soon as K(g) has landed and the softmax has read S(g-1);
-// then O += P(g-1) V(g-1) once P(g-1) is in TMEM.  The MMA pipe accepts one
-// tcgen05.mma every ~54-64 cycles, 12 per block: well inside the exponent
-// unit's ~1000 cycles per block, so one issuing thread is enough.
+// S(g) = Q K(g)^T into TMEM buffer g % 3 once K(g) has landed and the
+// product that last read that buffer, P(g - 3) V(g - 3), has finished; then
+// O += P(g-1) V(g-1) once P(g-1) is in TMEM.  Every product commits to the
+// O-complete barrier of its parity (two barriers, so a softmax thread that
+// only sometimes waits for a product can still tell the phases apart).
 __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                          volatile int* abort_flag, uint32_t tmem_base) {
-    const uint32_t idesc_s = idesc_bf16(kBM, kBN, 0, 0);
     const uint32_t idesc_pv = idesc_bf16(kBM, kHD, 0, 1);
-    uint64_t dQ[kStages], dK[kStages], dV[kStages];
+    uint64_t dQ[kQStages];
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) {
-        dQ[s] = sdesc_k_sw128(smem_u32(smem + kOffQ + s * kTileBytes));
-        dK[s] = sdesc_k_sw128(smem_u32(smem + kOffK + s * kTileBytes));
-        dV[s] = sdesc_mn_sw128(smem_u32(smem + kOffV + s * kTileBytes));
-    }
-    const uint32_t tS = tmem_base + kColS, tP = tmem_base + kColP, tO = tmem_base + kColO;
+    for (int st = 0; st < kQStages; ++st) dQ[st] = sdesc_k_sw128(smem_u32(smem + kOffQ + st * kQBytes));
+    const uint64_t dK0 = sdesc_k_sw128(smem_u32(smem + kOffK));
+    const uint64_t dV0 = sdesc_mn_sw128(smem_u32(smem + kOffV));
+    constexpr uint64_t kKVDescStep = kKVBytes >> 4;  // start-address units per ring stage
+    const uint32_t tO = tmem_base + kColO;
 
-    // O += P(g) V(g) over nk keys; the first block of a tile overwrites O
+    // O += P(g) V(g) over nk keys; the first block of a piece overwrites O
     auto issue_pv = [&](uint32_t g, int nk, bool first) -> bool {
-        const uint32_t s = g & 1u;
-        if (!mbar_wait(&bars[kBarPFull], g & 1u, abort_flag) ||
-            !mbar_wait(&bars[kBarVFull + s], (g >> 1) & 1u, abort_flag))
+        const uint32_t b = g % kSBufs, st = g % kKVStages;
+        if (!mbar_wait(&bars[kBarPFull + b], (g / kSBufs) & 1u, abort_flag, p.wait_ns) ||
+            !mbar_wait(&bars[kBarVFull + st], (g / kKVStages) & 1u, abort_flag, p.wait_ns))
             return false;
         tc_fence_after();
-        const uint64_t dv = dV[s];
-        if (nk == kBN) {
-            if (first)
-                tc_mma_ts<false>(tO, tP + 0, dv + 0, idesc_pv);
-            else
-                tc_mma_ts<true>(tO, tP + 0, dv + 0, idesc_pv);
-#pragma unroll
-            for (int k = 1; k < 8; ++k) tc_mma_ts<true>(tO, tP + 8u * k, dv + 128u * k, idesc_pv);
-        } else {  // a partial block of global keys (never the first block of a tile)
-            for (int k = 0; k < nk / 16; ++k) tc_mma_ts<true>(tO, tP + 8u * k, dv + 128u * k, idesc_pv);
-        }
-        tc_commit(&bars[kBarOFull]);
-        tc_commit(&bars[kBarVEmpty + s]);
+        const uint64_t dv = dV0 + kKVDescStep * st;
+        const uint32_t tP = tmem_base + 64u * b;
+        if (first)
+            tc_mma_ts<false>(tO, tP, dv, idesc_pv);
+        else
+            tc_mma_ts<true>(tO, tP, dv, idesc_pv);
+        for (int k = 1; k < nk / 16; ++k) tc_mma_ts<true>(tO, tP + 8u * k, dv + 128u * k, idesc_pv);
+        tc_commit(&bars[kBarBufFree + b]);
+        tc_commit(&bars[kBarOFull + (g & 1u)]);
+        tc_commit(&bars[kBarVEmpty + st]);
         return true;
     };
 
-    uint32_t g = 0, qt = 0, qs = 0;
-    int item = blockIdx.x, blk = 0, nb = 0, nbb = 0, ngk = 0;
+    uint32_t g = 0, qt = 0;
     int prev_nk = 0;
-    bool prev_first = false;
-    for (;;) {  // S(g), then the product of block g - 1
-        const bool have = item < p.n_items;
-        int cur_nk = 0;
-        bool cur_first = false;
-        if (have) {
-            if (blk == 0) {  // the tile's Q has landed and its descriptor is visible
-                qs = qt & 1u;
-                if (!mbar_wait(&bars[kBarQFull + qs], (qt >> 1) & 1u, abort_flag)) break;
-                ++qt;
-                const BandTile* d = reinterpret_cast<const BandTile*>(smem + kOffDesc + qs * kDescBytes);
-                nbb = d->nbb;
-                ngk = d->ngk;
-                nb = nbb + d->ngb;
-            }
-            const uint32_t s = g & 1u;
-            if (!mbar_wait(&bars[kBarKFull + s], (g >> 1) & 1u, abort_flag) ||
-                (g > 0 && !mbar_wait(&bars[kBarSFree], (g - 1) & 1u, abort_flag)))
+    bool prev_first = false, done = false;
+    while (!done) {
+        const uint32_t qs = qt & 1u;
+        if (!mbar_wait(&bars[kBarQFull + qs], (qt >> 1) & 1u, abort_flag, p.wait_ns)) break;
+        ++qt;
+        const BandPiece* d = reinterpret_cast<const BandPiece*>(smem + kOffDesc + qs * kDescBytes);
+        const int blk_lo = d->blk_lo, blk_hi = d->blk_hi, nbb = d->nbb, bsm = d->b;
+        int ngk = -1;  // global keys of this sample (prep's output), read at the first global block
+        done = d->last != 0;
+        bool ok = true;
+        for (int blk = blk_lo; blk < blk_hi; ++blk, ++g) {
+            const uint32_t b = g % kSBufs, st = g % kKVStages;
+            if (!mbar_wait(&bars[kBarKFull + st], (g / kKVStages) & 1u, abort_flag, p.wait_ns) ||
+                (g >= kSBufs && !mbar_wait(&bars[kBarBufFree + b], ((g / kSBufs) & 1u) ^ 1u, abort_flag, p.wait_ns))) {
+                ok = false;
                 break;
+            }
             tc_fence_after();
+            if (blk >= nbb && ngk < 0) {
+                grid_dep_wait();
+                ngk = *reinterpret_cast<const volatile int*>(p.n_gk + bsm);
+            }
             const int ncols = blk < nbb ? kBN : global_block_cols(ngk, blk - nbb);
-            const uint32_t ids = ncols == kBN ? idesc_s : idesc_bf16(kBM, ncols, 0, 0);
-            const uint64_t dq = dQ[qs], dk = dK[s];
+            const uint32_t ids = idesc_bf16(kBM, ncols, 0, 0);
+            const uint64_t dq = dQ[qs], dk = dK0 + kKVDescStep * st;
+            const uint32_t tS = tmem_base + 64u * b;
             tc_mma<false>(tS, dq + 0, dk + 0, ids);  // K-steps of 16 (32 bytes = 2 units)
             tc_mma<true>(tS, dq + 2, dk + 2, ids);
             tc_mma<true>(tS, dq + 4, dk + 4, ids);
             tc_mma<true>(tS, dq + 6, dk + 6, ids);
-            tc_commit(&bars[kBarSFull]);
-            tc_commit(&bars[kBarKEmpty + s]);
-            if (blk == nb - 1) tc_commit(&bars[kBarQEmpty + qs]);
-            cur_nk = ncols;
-            cur_first = blk == 0;
+            tc_commit(&bars[kBarSFull + b]);
+            tc_commit(&bars[kBarKEmpty + st]);
+            if (blk == blk_hi - 1) tc_commit(&bars[kBarQEmpty + qs]);
+            if (g > 0 && !issue_pv(g - 1, prev_nk, prev_first)) {
+                ok = false;
+                break;
+            }
+            prev_nk = ncols;
+            prev_first = blk == blk_lo;
         }
-        if (g > 0 && !issue_pv(g - 1, prev_nk, prev_first)) break;
-        if (!have) break;
-        prev_nk = cur_nk;
-        prev_first = cur_first;
-        ++g;
-        if (++blk == nb) {
-            blk = 0;
-            item += gridDim.x;
-        }
+        if (!ok) break;
+        if (done && g > 0) (void)issue_pv(g - 1, prev_nk, prev_first);
     }
     tc_commit(&bars[kBarDrain]);
 }
 
 // ------------------------------------------------------------ softmax role
-// Thread x owns query row x of the tile (TMEM lane x) and walks each S block
-// in four chunks of 32 columns, one loop body for all of them: TMEM load,
-// mask, max, exponentials, P (16 columns of bf16 pairs) back to TMEM, so
-// only one chunk of S is held in registers.
-//
-// Exponent base.  p = 2^(s*sl2 - base) with base = m_ref.  The base moves
-// between blocks, to the largest scaled score seen so far, once that exceeds
-// it by more than 2^8 (O and the row sum are rescaled then; the O rescale
-// needs the previous product to have finished, which the P store waits for
-// anyway).  Inside a block the base stays put unless a chunk's max exceeds
-// it by more than 2^64, so p < 2^64 and fp32 sums stay finite; that rare
-// jump rescales O and the P chunks already stored.
-constexpr float kBigJumpLog2 = 64.f;
+// Thread x owns query row x of the tile (TMEM lane x).  Per block: wait for
+// S, load the row's 64 scores, mask, take the block max, move the exponent
+// base if needed, exponentiate, store P over S.  The output (or partial
+// state) of a piece is written when the next piece starts, or at the end,
+// once the piece's last product has finished.
 
-// Multiplies the first nchunks P chunks (16 columns of bf16 pairs each) of
-// this thread's row by alpha, in TMEM.
-__device__ __forceinline__ void rescale_p_chunks(uint32_t tP, int nchunks, float alpha) {
-    tmem_st_wait();  // this thread's own stores have landed
-#pragma unroll 1
-    for (int c = 0; c < nchunks; ++c) {
-        uint32_t pr[16];
-        tmem_ld16(tP + 16u * c, pr);
-        tmem_ld_wait16(pr);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&pr[u]);
-            const float2 f = __bfloat1622float2(h);
-            pr[u] = pack_bf16x2(f.x * alpha, f.y * alpha);
-        }
-        tmem_st16(tP + 16u * c, pr);
-    }
-}
-
-// Multiplies this thread's row of O (64 fp32 columns) by alpha, in TMEM.
-__device__ __noinline__ void rescale_o(uint32_t tO, float alpha) {
-#pragma unroll 1
-    for (int part = 0; part < 4; ++part) {
-        uint32_t orr[16];
-        tmem_ld16(tO + 16u * part, orr);
-        tmem_ld_wait16(orr);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-        tmem_st16(tO + 16u * part, orr);
-    }
-}
-
-// Writes this thread's output row, y = O * inv as bf16 (dst null: row not
-// written), from TMEM.  Once per tile, out of line.
-__device__ __noinline__ void write_rows(uint32_t tO, uint4* dst, float inv) {
+// Multiplies this thread's row of O (64 fp32 columns) by alpha, in TMEM,
+// 16 columns at a time (few registers: it runs inside the block loop).
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 #pragma unroll 1
     for (int part = 0; part < 4; ++part) {
         uint32_t o[16];
         tmem_ld16(tO + 16u * part, o);
         tmem_ld_wait16(o);
-        if (dst) {
-            uint4 v0, v1;
-            v0.x = pack_bf16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
-            v0.y = pack_bf16x2(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
-            v0.z = pack_bf16x2(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
-            v0.w = pack_bf16x2(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
-            v1.x = pack_bf16x2(__uint_as_float(o[8]) * inv, __uint_as_float(o[9]) * inv);
-            v1.y = pack_bf16x2(__uint_as_float(o[10]) * inv, __uint_as_float(o[11]) * inv);
-            v1.z = pack_bf16x2(__uint_as_float(o[12]) * inv, __uint_as_float(o[13]) * inv);
-            v1.w = pack_bf16x2(__uint_as_float(o[14]) * inv, __uint_as_float(o[15]) * inv);
-            dst[2 * part] = v0;
-            dst[2 * part + 1] = v1;
-        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+        tmem_st16(tO + 16u * part, o);
     }
 }
 
-// Rare path of a score jump inside a block: multiplies the first nchunks P
-// chunks of this thread's row, and (with_o) its row of O, by alpha, in TMEM.
-__device__ __noinline__ void rescale_held(uint32_t tP, int nchunks, uint32_t tO, bool with_o, float alpha) {
-    rescale_p_chunks(tP, nchunks, alpha);
-    if (with_o) rescale_o(tO, alpha);
+// Writes y = O * inv as bf16 to dst (16-byte stores).
+__device__ __forceinline__ void store_row(__nv_bfloat16* dst, const float* o, float inv) {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        uint4 v;
+        v.x = pack_bf16x2(o[8 * u + 0] * inv, o[8 * u + 1] * inv);
+        v.y = pack_bf16x2(o[8 * u + 2] * inv, o[8 * u + 3] * inv);
+        v.z = pack_bf16x2(o[8 * u + 4] * inv, o[8 * u + 5] * inv);
+        v.w = pack_bf16x2(o[8 * u + 6] * inv, o[8 * u + 7] * inv);
+        d4[u] = v;
+    }
 }
 
-__device__ __forceinline__ uint32_t pick4(const uint32_t* v, int c) {
-    return c == 0 ? v[0] : (c == 1 ? v[1] : (c == 2 ? v[2] : v[3]));
+// Partial slot of CTA s's piece of a tile that starts at tstart: 2s for the
+// piece at the start of s's range, 2s + 1 for the one at its end.
+__device__ __forceinline__ float* part_slot(const BandTcParams& p, int s, int tstart) {
+    const int k = 2 * s + (tstart > range_start(p, s) ? 1 : 0);
+    return p.part + static_cast<size_t>(k) * kPartFloats;
+}
+
+// Output of a finished piece (warp-wide: every lane calls it): its
+// descriptor d stays in shared memory until this is done; m and l are this
+// thread's row's exponent base and sum.
+__device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiece* d, float m, float l, uint32_t tO,
+                                          int wq, int ticket, volatile int* abort_flag) {
+    const int lane = threadIdx.x & 31;
+    const int x = wq * 32 + lane;
+    const int self = static_cast<int>(blockIdx.x);
+    const int ip = d->q0 + x, Tc = d->Tc;
+    const int i = d->c + d->dil * ip;
+    bool write = ip < Tc;
+    if (write) write = !((p.gbit[static_cast<size_t>(d->b) * p.W + (i >> 5)] >> (i & 31)) & 1u);
+    __nv_bfloat16* dst = p.out + (static_cast<size_t>(d->bh) * p.T + (write ? i : 0)) * kHD;
+    float o[64];
+    {
+        uint32_t r[64];
+        tmem_ld64(tO, r);
+        tmem_ld_wait(r);
+        reg_fence32(r + 32);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) o[c] = __uint_as_float(r[c]);
+    }
+    if (d->blk_lo == 0 && d->blk_hi == d->nbb + d->ngb) {  // the whole tile
+        if (write) store_row(dst, o, l > 0.f ? 1.f / l : 0.f);
+        return;
+    }
+    const int s0 = d->s0, s1 = d->s1;
+    const int tstart = d->tstart;
+    int* cnt = p.cnt + (static_cast<size_t>(d->tile) * 4 + wq) * 2;  // [0] arrivals, [1] lanes done writing
+    const int npieces = s1 - s0 + 1;
+    if (ticket < npieces - 1) {  // not the last to arrive: leave the partial state for the last
+        float* slot = part_slot(p, self, tstart);
+        float4* o4 = reinterpret_cast<float4*>(slot);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) o4[u * kBM + x] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        slot[kBM * kHD + x] = m;
+        slot[kBM * kHD + kBM + x] = l;
+        red_release_add(cnt + 1, 1);  // each lane: its stores, then its count (no wait)
+        return;
+    }
+    // the last to arrive: the others arrived earlier and write without waiting
+    // for anything; every lane acquires their count, so their partial states
+    // are visible to it
+    bool ok = true;
+    {
+        const int want = 32 * (npieces - 1);
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t it = 0; __any_sync(0xffffffffu, ld_acquire(cnt + 1) < want); ++it) {
+            if ((it & 63u) == 63u && globaltimer_ns() - t0 > p.wait_ns) {
+                if (lane == 0) *abort_flag = 1;
+                ok = false;
+                break;
+            }
+        }
+    }
+    // M = max of the pieces' bases; y = sum_s w_s O_s / sum_s w_s l_s with w_s = 2^(m_s - M),
+    // summed in CTA order whichever piece merges (the same operations either way)
+    float acc[64];
+    float L = 0.f;
+    if (npieces == 2 && ok) {  // the common case: one other piece, all its loads at once
+        const int so = self == s0 ? s1 : s0;
+        const float* slot = part_slot(p, so, tstart);
+        const float4* o4 = reinterpret_cast<const float4*>(slot);
+        float4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] = __ldcg(o4 + u * kBM + x);
+        const float mo = __ldcg(slot + kBM * kHD + x);
+        const float lo = __ldcg(slot + kBM * kHD + kBM + x);
+        const float M = fmaxf(m, mo);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        const float ws = m == -INFINITY ? 0.f : ex2_approx(m - Mu);
+        const float wo = mo == -INFINITY ? 0.f : ex2_approx(mo - Mu);
+        const bool self_first = self == s0;
+        const float w1 = self_first ? ws : wo, w2 = self_first ? wo : ws;
+        L = fmaf(w2, self_first ? lo : l, w1 * (self_first ? l : lo));
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const float a0 = v[u].x, a1 = v[u].y, a2 = v[u].z, a3 = v[u].w;
+            const float b0 = o[4 * u], b1 = o[4 * u + 1], b2 = o[4 * u + 2], b3 = o[4 * u + 3];
+            acc[4 * u] = fmaf(w2, self_first ? a0 : b0, w1 * (self_first ? b0 : a0));
+            acc[4 * u + 1] = fmaf(w2, self_first ? a1 : b1, w1 * (self_first ? b1 : a1));
+            acc[4 * u + 2] = fmaf(w2, self_first ? a2 : b2, w1 * (self_first ? b2 : a2));
+            acc[4 * u + 3] = fmaf(w2, self_first ? a3 : b3, w1 * (self_first ? b3 : a3));
+        }
+    } else {
+        float M = m;
+        for (int s = s0; s <= s1; ++s)
+            if (s != self && ok) M = fmaxf(M, __ldcg(part_slot(p, s, tstart) + kBM * kHD + x));
+        const float Mu = M == -INFINITY ? 0.f : M;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+        for (int s = s0; s <= s1; ++s) {
+            if (s == self) {
+                const float wv = m == -INFINITY ? 0.f : ex2_approx(m - Mu);
+                L = fmaf(wv, l, L);
+#pragma unroll
+                for (int c = 0; c < 64; ++c) acc[c] = fmaf(wv, o[c], acc[c]);
+                continue;
+            }
+            if (!ok) continue;
+            const float* slot = part_slot(p, s, tstart);
+            const float ms = __ldcg(slot + kBM * kHD + x);
+            const float wv = ms == -INFINITY ? 0.f : ex2_approx(ms - Mu);
+            L = fmaf(wv, __ldcg(slot + kBM * kHD + kBM + x), L);
+            const float4* o4 = reinterpret_cast<const float4*>(slot);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const float4 v = __ldcg(o4 + u * kBM + x);
+                acc[4 * u] = fmaf(wv, v.x, acc[4 * u]);
+                acc[4 * u + 1] = fmaf(wv, v.y, acc[4 * u + 1]);
+                acc[4 * u + 2] = fmaf(wv, v.z, acc[4 * u + 2]);
+                acc[4 * u + 3] = fmaf(wv, v.w, acc[4 * u + 3]);
+            }
+        }
+    }
+    if (write) store_row(dst, acc, L > 0.f ? 1.f / L : 0.f);
+    __syncwarp();
+    if (lane == 0) {  // ready for the next call
+        cnt[0] = 0;
+        cnt[1] = 0;
+    }
 }
 
 __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
@@ -431,222 +669,234 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     const int wq = warp & 3;
     const int x = wq * 32 + lane;  // query row inside the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem_base + lane_off + kColS;
-    const uint32_t tP = tmem_base + lane_off + kColP;
     const uint32_t tO = tmem_base + lane_off + kColO;
     // scale >= 0: maxima on raw scores (masked columns -inf); scale < 0: minima
     // (masked columns +inf); either way the scale is folded into the exp2 FMA
     const bool pos = p.sl2 >= 0.f;
     const float kmul = p.sl2 == 0.f ? 1e-30f : p.sl2;
     const uint32_t fill = __float_as_uint(pos ? -INFINITY : INFINITY);
-    uint32_t g = 0;
+    // prep's output (global-key lists and counts, the global-row bitmap, the
+    // zeroed merge tickets) is needed only from the first global-key block or
+    // the first rows written; the band blocks before that overlap prep
+    bool prep_done = false;
+    auto need_prep = [&]() {
+        if (!prep_done) {
+            grid_dep_wait();
+            prep_done = true;
+        }
+    };
 
     // every lane polls (each lane's own acquire), then the warp agrees on the outcome
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
-        const bool ok = mbar_wait(bar, parity, abort_flag);
+        const bool ok = mbar_wait(bar, parity, abort_flag, p.wait_ns);
         return __all_sync(0xffffffffu, ok);
     };
-
-    // The output row of a finished tile is written once the product that
-    // completes its O is done, which the first P store of the next tile (or
-    // the end of the role) waits for anyway.
-    bool pend = false, pend_ok = false;
-    float pend_inv = 0.f;
-    uint4* pend_dst = nullptr;
-    auto flush = [&]() {
-        if (!pend) return;
-        pend = false;
-        write_rows(tO, pend_ok ? pend_dst : nullptr, pend_inv);
+    // the product of block gp has finished (the O-complete barrier of its parity)
+    auto wait_product = [&](uint32_t gp) -> bool {
+        if (!wait_warp(&bars[kBarOFull + (gp & 1u)], (gp >> 1) & 1u)) return false;
+        tc_fence_after();
+        return true;
     };
 
-    uint32_t qt = 0;
-    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-        // the tile's descriptor, published by the producer with its Q tile
+    // this CTA's current sample's global keys: count and the first 64 (lane a
+    // holds keys a and 32 + a), loaded at the first global block of a sample
+    int gk_b = -1, ngk = 0;
+    uint32_t gk_reg[2] = {0u, 0u};
+
+    uint32_t g = 0, qt = 0;
+    bool done = false;
+    // The previous piece, until its last product is done and its rows are
+    // written; its descriptor slot is released (Q-empty) only then.
+    int prev_slot = -1;
+    float m_prev = 0.f, l_prev = 0.f;
+    int ticket = 0;  // merge ticket of the previous piece (split pieces)
+    auto finish_prev = [&]() {
+        const BandPiece* dq = reinterpret_cast<const BandPiece*>(smem + kOffDesc + prev_slot * kDescBytes);
+        flush_rows(p, dq, m_prev, l_prev, tO, wq, __shfl_sync(0xffffffffu, ticket, 0), abort_flag);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarQEmpty + prev_slot]);
+        prev_slot = -1;
+    };
+    for (;;) {
+        // the previous piece's O is final once its last product is done: its rows
+        // (one place in the code for every piece, the last one included)
+        if (prev_slot >= 0) {
+            if (!wait_product(g - 1)) return;
+            need_prep();
+            finish_prev();
+        }
+        if (done) break;
+        // the piece's descriptor, published by the producer with its Q tile
         const uint32_t qs = qt & 1u;
         if (!wait_warp(&bars[kBarQFull + qs], (qt >> 1) & 1u)) return;
         ++qt;
-        const BandTile t = *reinterpret_cast<const BandTile*>(smem + kOffDesc + qs * kDescBytes);
-        const int ip = t.q0 + x;         // decimated row index
-        const int i = t.c + t.dil * ip;  // position in the sequence
-        // global-row bitmap word of this row; consumed only when the tile's rows are written
-        const uint32_t gbw = ip < t.Tc ? __ldg(p.gbit + static_cast<size_t>(t.b) * p.W + (i >> 5)) : 0u;
-        const int32_t* gk = p.gk_list + static_cast<size_t>(t.b) * p.gstride;
-        const int reach = t.dil * p.r;
-        // the first block of global keys, one key per lane and chunk, fetched early
-        uint32_t kreg[4] = {0u, 0u, 0u, 0u};
-        if (t.ngb > 0) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-                if (32 * w + lane < t.ngk) kreg[w] = static_cast<uint32_t>(__ldg(gk + 32 * w + lane));
+        const BandPiece* dp = reinterpret_cast<const BandPiece*>(smem + kOffDesc + qs * kDescBytes);
+        done = dp->last != 0;
+        const int blk_lo = dp->blk_lo, blk_hi = dp->blk_hi, nbb = dp->nbb;
+        const int i = dp->c + dp->dil * (dp->q0 + x);  // this row's position in the sequence
+        // Band blocks inside every row's window and inside [0, Tc) need no mask:
+        // 0 <= 64 kb + y - x <= 2r for all x < 128, y < 64, and 0 <= j0, j0 + 64 <= Tc.
+        int ib_lo = nbb, ib_hi = nbb;
+        if (!p.pad) {
+            const int kb_a = max(2, (-dp->kbase + kBN - 1) / kBN);
+            const int kb_b = min((2 * p.r - kBN + 1) / kBN, (dp->Tc - kBN - dp->kbase) >= 0 ? (dp->Tc - kBN - dp->kbase) / kBN : -1);
+            if (kb_b >= kb_a) {
+                ib_lo = max(0, kb_a - dp->kb_lo);
+                ib_hi = min(nbb, kb_b + 1 - dp->kb_lo);
+            }
         }
+        const bool split = blk_lo > 0 || blk_hi < nbb + dp->ngb;
 
-        float m_ref = -INFINITY;   // exponent base (scaled, log2 domain; -inf: nothing valid yet)
-        float m_seen = -INFINITY;  // largest scaled score seen so far
-        float l_row = 0.f;         // row sum relative to m_ref
-        const int nb = t.nbb + t.ngb;
-        for (int blk = 0; blk < nb; ++blk, ++g) {
-            // ---- which columns this row keeps: band blocks inside every row's window and
-            //      inside [0, Tc) need no test (128 kb + y - x lies in [0, 2r] for all x, y)
-            const bool band = blk < t.nbb;
-            const int kb = t.kb_lo + blk;
-            const int j0 = t.kbase + kBN * kb;
-            const bool interior =
-                band && !p.pad && kb >= 1 && kBN * kb + kBN - 1 <= 2 * p.r && j0 >= 0 && j0 + kBN <= t.Tc;
-            const int ylo = max(max(0, x - kBN * kb), -j0);  // band: kept columns [ylo, yhi)
-            const int yhi = min(min(kBN, x + 2 * p.r + 1 - kBN * kb), t.Tc - j0);
-            uint32_t padv[4] = {0u, 0u, 0u, 0u};  // band: key padding of column 32 w + lane
-            int nch = 4, nvalid = kBN;
-            if (band) {
-                if (p.pad) {
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const int jd = j0 + 32 * w + lane;
-                        if (jd >= 0 && jd < t.Tc)
-                            padv[w] = p.pad[static_cast<size_t>(t.b) * p.T + t.c + static_cast<size_t>(t.dil) * jd];
-                    }
-                }
-            } else {
-                const int gb = blk - t.nbb;
-                nvalid = min(kBN, t.ngk - gb * kBN);
-                nch = (nvalid + 31) >> 5;
-                if (gb > 0) {
-#pragma unroll
-                    for (int w = 0; w < 4; ++w)
-                        kreg[w] = 32 * w + lane < nvalid ? static_cast<uint32_t>(__ldg(gk + gb * kBN + 32 * w + lane)) : 0u;
-                }
-            }
-
-            // ---- deferred base move (decided on the blocks before this one)
-            float alpha_o = 1.f;
-            const bool o_move = m_ref != -INFINITY && m_seen > m_ref + kRescaleLog2;
-            if (o_move) {
-                alpha_o = ex2_approx(m_ref - m_seen);
-                m_ref = m_seen;
-                l_row *= alpha_o;
-            }
-            const bool warp_o_move = __any_sync(0xffffffffu, o_move);
-            // P may be overwritten (and O touched) once the previous product is done
-            bool p_ready = false;
-            auto ensure_p_ready = [&]() -> bool {
-                if (p_ready) return true;
-                if (g > 0) {
-                    if (!wait_warp(&bars[kBarOFull], (g - 1) & 1u)) return false;
-                    tc_fence_after();
-                }
-                flush();
-                if (warp_o_move) rescale_o(tO, alpha_o);
-                p_ready = true;
-                return true;
-            };
-
-            if (!wait_warp(&bars[kBarSFull], g & 1u)) return;
-            tc_fence_after();
-            float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-            // one body for every chunk: a second copy (for a load in flight during the
-            // previous chunk) costs more in instruction fetch than it hides
+        float m_ref = -INFINITY;  // exponent base (scaled, log2 domain; -inf: nothing kept yet)
+        float l_row = 0.f;        // row sum relative to m_ref
 #pragma unroll 1
-            for (int c = 0; c < nch; ++c) {
-                uint32_t cur[32];
-                tmem_ld32(tS + 32u * c, cur);
-                tmem_ld_wait(cur);
-                if (c + 1 == nch) {  // the whole S block has been read: the MMA may overwrite it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars[kBarSFree]);
-                }
-                if (!interior) {
-                    uint32_t m;
-                    if (band) {
-                        m = range_bits(ylo - 32 * c, yhi - 32 * c);
-                        if (p.pad) m &= ~__ballot_sync(0xffffffffu, pick4(padv, c) != 0u);
-                    } else {  // global keys not already in the row's window
-                        m = 0u;
-                        const uint32_t kc = pick4(kreg, c);
-                        const int na = min(32, nvalid - 32 * c);
-#pragma unroll 1
-                        for (int a = 0; a < na; ++a) {
-                            const int diff = static_cast<int>(__shfl_sync(0xffffffffu, kc, a)) - i;
-                            const bool in_window =
-                                diff <= reach && diff >= -reach && (t.dil == 1 || diff % t.dil == 0);
-                            m |= in_window ? 0u : (1u << a);
+        for (int blk = blk_lo; blk < blk_hi; ++blk, ++g) {
+            const uint32_t b = g % kSBufs;
+            // ---- which columns this row keeps (bit j of mk[c]: column 32 c + j)
+            uint32_t mk[2] = {0xffffffffu, 0xffffffffu};
+            bool live0 = true, live1 = true, full0 = true, full1 = true;
+            if (blk < ib_lo || blk >= ib_hi) {
+                if (blk < nbb) {
+                    const int kb = dp->kb_lo + blk;
+                    const int Tc = dp->Tc;
+                    const int j0 = dp->kbase + kBN * kb;
+                    // kept columns [ylo, yhi): the window and [0, Tc)
+                    const int ylo = max(max(0, x - kBN * kb), -j0);
+                    const int yhi = min(min(kBN, x + 2 * p.r + 1 - kBN * kb), Tc - j0);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t m = range_bits(ylo - 32 * c, yhi - 32 * c);
+                        if (p.pad) {
+                            const int jd = j0 + 32 * c + lane;
+                            const bool padded =
+                                jd >= 0 && jd < Tc &&
+                                p.pad[static_cast<size_t>(dp->b) * p.T + dp->c + static_cast<size_t>(dp->dil) * jd] != 0;
+                            m &= ~__ballot_sync(0xffffffffu, padded);
                         }
+                        mk[c] = m;
                     }
-                    if (!__all_sync(0xffffffffu, m == 0xffffffffu)) {  // only chunks some row masks
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (!((m >> j) & 1u)) cur[j] = fill;
+                } else {  // global keys not already in the row's window
+                    const int bs = dp->b;
+                    if (bs != gk_b) {
+                        need_prep();
+                        gk_b = bs;
+                        ngk = *reinterpret_cast<const volatile int*>(p.n_gk + bs);
+                        const int32_t* gl = p.gk_list + static_cast<size_t>(bs) * p.gstride;
+                        gk_reg[0] = lane < ngk ? static_cast<uint32_t>(gl[lane]) : 0u;
+                        gk_reg[1] = 32 + lane < ngk ? static_cast<uint32_t>(gl[32 + lane]) : 0u;
                     }
-                }
-                float mx;
-                if (pos) {
-                    float mxp[4];
+                    const int gb = blk - nbb;
+                    const int nvalid = min(kBN, ngk - gb * kBN);
+                    const int32_t* gkl = p.gk_list + static_cast<size_t>(bs) * p.gstride + gb * kBN;
+                    const int dil = dp->dil, reach = dil * p.r;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) mxp[u] = fmaxf(__uint_as_float(cur[2 * u]), __uint_as_float(cur[2 * u + 1]));
-#pragma unroll
-                    for (int j = 8; j < 32; j += 8)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            mxp[u] = fmax3(mxp[u], __uint_as_float(cur[j + 2 * u]), __uint_as_float(cur[j + 2 * u + 1]));
-                    mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
-                } else {
-                    float mnp[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) mnp[u] = fminf(__uint_as_float(cur[2 * u]), __uint_as_float(cur[2 * u + 1]));
-#pragma unroll
-                    for (int j = 8; j < 32; j += 8)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            mnp[u] = fmin3(mnp[u], __uint_as_float(cur[j + 2 * u]), __uint_as_float(cur[j + 2 * u + 1]));
-                    mx = fminf(fminf(mnp[0], mnp[1]), fminf(mnp[2], mnp[3]));
-                }
-                mx *= kmul;  // the largest scaled score of the chunk (-inf if none is kept)
-                m_seen = fmaxf(m_seen, mx);
-                if (m_ref == -INFINITY) m_ref = mx;  // everything so far had zero weight
-                const bool big = mx > m_ref + kBigJumpLog2;
-                if (__any_sync(0xffffffffu, big)) {  // rare: rescale what this block already holds
-                    const float alpha = big ? ex2_approx(m_ref - mx) : 1.f;
-                    if (big) {
-                        m_ref = mx;
-                        l_row *= alpha;
-                        lsum[0] *= alpha;
-                        lsum[1] *= alpha;
-                        lsum[2] *= alpha;
-                        lsum[3] *= alpha;
-                    }
-                    if (c > 0 || blk > 0) {
-                        if (!ensure_p_ready()) return;
-                        rescale_held(tP, c, tO, blk > 0, alpha);
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t m = 0u;
+                        const int na = min(32, nvalid - 32 * c);
+                        if (na > 0) {
+                            const uint32_t kc = gb == 0 ? gk_reg[c] : (lane < na ? static_cast<uint32_t>(gkl[32 * c + lane]) : 0u);
+#pragma unroll 1
+                            for (int a = 0; a < na; ++a) {
+                                const int diff = static_cast<int>(__shfl_sync(0xffffffffu, kc, a)) - i;
+                                const bool in_window = diff <= reach && diff >= -reach && (dil == 1 || diff % dil == 0);
+                                m |= in_window ? 0u : (1u << a);
+                            }
+                        }
+                        mk[c] = m;
                     }
                 }
-                const float nb2 = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                uint32_t pk[16];
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const float e0 = ex2_approx(fmaf(__uint_as_float(cur[j]), kmul, nb2));
-                    const float e1 = ex2_approx(fmaf(__uint_as_float(cur[j + 1]), kmul, nb2));
-                    lsum[(j >> 1) & 3] += e0 + e1;
-                    pk[j >> 1] = pack_bf16x2(e0, e1);
-                }
-                // the previous product is waited for only here, after chunk 0's work
-                if (c == 0 && !ensure_p_ready()) return;
-                tmem_st16(tP + 16u * c, pk);
+                live0 = __any_sync(0xffffffffu, mk[0] != 0u);
+                live1 = __any_sync(0xffffffffu, mk[1] != 0u);
+                full0 = __all_sync(0xffffffffu, mk[0] == 0xffffffffu);
+                full1 = __all_sync(0xffffffffu, mk[1] == 0xffffffffu);
             }
-            l_row += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+
+            if (split && blk == blk_hi - 1) {  // the merge ticket, while this last block is computed
+                need_prep();                     // (prep zeroes the tickets)
+                if (lane == 0) ticket = atomicAdd(p.cnt + (static_cast<size_t>(dp->tile) * 4 + wq) * 2, 1);
+            }
+
+            // ---- the row's 64 scores
+            if (!wait_warp(&bars[kBarSFull + b], (g / kSBufs) & 1u)) return;
+            tc_fence_after();
+            const uint32_t tS = tmem_base + lane_off + 64u * b;
+            uint32_t s[64];
+            tmem_ld64(tS, s);
+            tmem_ld_wait(s);
+            reg_fence32(s + 32);
+
+            // ---- mask and block max (scaled: the largest kept s * kmul)
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+            if (live0) {
+                if (!full0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (!((mk[0] >> j) & 1u)) s[j] = fill;
+                }
+                mx0 = (pos ? max32(s) : min32(s)) * kmul;
+            }
+            if (live1) {
+                if (!full1) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (!((mk[1] >> j) & 1u)) s[32 + j] = fill;
+                }
+                mx1 = (pos ? max32(s + 32) : min32(s + 32)) * kmul;
+            }
+            const float mxs = fmaxf(mx0, mx1);
+            // ---- exponent base
+            float alpha = 1.f;
+            bool o_move = false;
+            if (m_ref == -INFINITY) {
+                m_ref = mxs;  // nothing held so far (the row's O and l are 0)
+            } else if (mxs > m_ref + kRescaleLog2) {
+                alpha = ex2_approx(m_ref - mxs);
+                l_row *= alpha;
+                m_ref = mxs;
+                o_move = true;
+            }
+            const float nb2 = m_ref == -INFINITY ? 0.f : -m_ref;
+
+            // ---- p = 2^(s * kmul - base), row sums, bf16 pairs
+            uint32_t pk[32];
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+            const float2 k2 = make_float2(kmul, kmul), b2 = make_float2(nb2, nb2);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                if (c == 0 ? live0 : live1) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float2 t0 = ffma2(make_float2(__uint_as_float(s[32 * c + j]), __uint_as_float(s[32 * c + j + 1])), k2, b2);
+                        const float2 t1 = ffma2(make_float2(__uint_as_float(s[32 * c + j + 2]), __uint_as_float(s[32 * c + j + 3])), k2, b2);
+                        const float2 e0 = make_float2(ex2_approx(t0.x), ex2_approx(t0.y));
+                        const float2 e1 = make_float2(ex2_approx(t1.x), ex2_approx(t1.y));
+                        acc0 = fadd2(acc0, e0);
+                        acc1 = fadd2(acc1, e1);
+                        pk[16 * c + j / 2] = pack_bf16x2(e0.x, e0.y);
+                        pk[16 * c + j / 2 + 1] = pack_bf16x2(e1.x, e1.y);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) pk[16 * c + j] = 0u;
+                }
+            }
+            l_row += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+
+            // ---- P over S; O is rescaled only once the previous product is done
+            tmem_st32(tS, pk);
+            if (__any_sync(0xffffffffu, o_move)) {
+                if (!wait_product(g - 1)) return;
+                rescale_o(tO, alpha);
+            }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kBarPFull]);
+            if (lane == 0) mbar_arrive(&bars[kBarPFull + b]);
         }
-        // ---- this tile's rows: y = O / l, written once its last product is done
-        pend = true;
-        pend_ok = ip < t.Tc && !((gbw >> (i & 31)) & 1u);
-        pend_inv = l_row > 0.f ? 1.f / l_row : 0.f;
-        pend_dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t.bh) * p.T + i) * kHD);
-    }
-    if (g > 0) {
-        if (!wait_warp(&bars[kBarOFull], (g - 1) & 1u)) return;
-        tc_fence_after();
-        flush();
+        // ---- this piece's rows are written once its last product is done
+        prev_slot = static_cast<int>(qs);
+        m_prev = m_ref;
+        l_prev = l_row;
     }
 }
 
@@ -662,18 +912,23 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kQStages; ++s) {
             mbar_init(&bars[kBarQFull + s], 1);
-            mbar_init(&bars[kBarQEmpty + s], 1);
+            mbar_init(&bars[kBarQEmpty + s], 1 + kSoftmaxWarps);  // last product of the piece + its rows written
+        }
+        for (int s = 0; s < kKVStages; ++s) {
             mbar_init(&bars[kBarKFull + s], 1);
             mbar_init(&bars[kBarKEmpty + s], 1);
             mbar_init(&bars[kBarVFull + s], 1);
             mbar_init(&bars[kBarVEmpty + s], 1);
         }
-        mbar_init(&bars[kBarSFull], 1);
-        mbar_init(&bars[kBarSFree], kSoftmaxWarps);
-        mbar_init(&bars[kBarPFull], kSoftmaxWarps);
+        for (int s = 0; s < kSBufs; ++s) {
+            mbar_init(&bars[kBarSFull + s], 1);
+            mbar_init(&bars[kBarPFull + s], kSoftmaxWarps);
+            mbar_init(&bars[kBarBufFree + s], 1);
+        }
         mbar_init(&bars[kBarOFull], 1);
+        mbar_init(&bars[kBarOFull + 1], 1);
         mbar_init(&bars[kBarDrain], 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -695,14 +950,23 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // the set-up above may overlap the prep kernel; its lists and packed keys are read below
-    grid_dep_wait();
 
+    // The set-up above may overlap the prep kernel; each role waits for it
+    // (griddepcontrol.wait) before it reads prep's output.
     if (warp == 0) {
         if (lane == 0) producer_role(p, smem, bars, abort_flag);
     } else if (warp == 1) {
         if (lane == 0) mma_role(p, smem, bars, abort_flag, tmem_base);
     } else {
+        {  // touch every 64-byte line of the parameters once, so the producer's walk hits in cache
+            const int t = threadIdx.x - 64;
+            constexpr int kLines = (sizeof(BandTcParams) + 63) / 64;
+            if (t < kLines) {
+                int v;
+                memcpy(&v, reinterpret_cast<const char*>(&p) + 64 * t, sizeof(int));
+                asm volatile("" ::"r"(v));
+            }
+        }
         softmax_role(p, smem, bars, abort_flag, tmem_base);
     }
 

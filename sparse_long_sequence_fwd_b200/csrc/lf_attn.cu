@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -46,25 +47,28 @@ struct DeviceState {
     static constexpr int kMaxSlices = 8;
     cudaStream_t cin = nullptr, cout = nullptr;
     cudaEvent_t ev_in[kMaxSlices] = {}, ev_done[kMaxSlices] = {};
-    // Band work items in longest-first order (device copy), for the shape in
-    // order_key; rebuilt outside stream capture when the shape changes.
-    bool may_order = true;  // false: never allocate for it (the allocation-free entry point)
-    int32_t* order = nullptr;
-    size_t order_cap = 0;
-    bool order_identity = true;
-    std::vector<int> order_key;
 };
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 thread_local int t_last_launches = 0;
+// Test hooks (lf_attn_test_hooks): the band kernel's pipeline-wait limit
+// (0: LF_WAIT_NS) and whether its producers stop before their first load.
+std::atomic<unsigned long long> g_test_wait_ns{0};
+std::atomic<int> g_test_stall{0};
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Band kernel: at most this many CTAs (two per SM of a 148-SM B200; larger
+// GPUs run it on 296 CTAs too), so its partial-state region has a size
+// known without a device.
+constexpr int kMaxBandCtas = 296;
+
 struct Layout {
-    size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, total;
+    size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, off_bcnt, off_bpart, total;
     int W, gstride, nchunk, ngp, cpc;  // nchunk: partial states per global row
+    long long band_tiles;             // upper bound on the band kernel's tiles (its merge tickets)
 };
 
 Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
@@ -98,6 +102,15 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
         const size_t kgb = sizeof(__nv_bfloat16) * size_t(B) * H * L.ngp * 64;
         L.off_vg = align256(o + kgb);
         o = align256(L.off_vg + kgb);
+    }
+    L.off_bcnt = o;
+    L.off_bpart = o;
+    L.band_tiles = 0;
+    if (dtype == LF_BF16) {
+        // every head has at most ceil(T / 128) + kMaxDilTma - 1 tiles (one per residue class more)
+        L.band_tiles = (long long)B * H * ((T + kBM - 1) / kBM + kMaxDilTma - 1);
+        L.off_bpart = align256(o + sizeof(int32_t) * size_t(L.band_tiles) * 8);
+        o = align256(L.off_bpart + sizeof(float) * size_t(2 * kMaxBandCtas) * kPartFloats);
     }
     L.total = std::max<size_t>(o, 256);
     return L;
@@ -238,6 +251,82 @@ lf_status check_args(const void* q, const void* k, const void* v, void* out, int
     return LF_OK;
 }
 
+// Groups the heads by dilation (one set of tensor maps per distinct value).
+int assign_kinds(BandTcParams& bp, int H, const int32_t* dil, int* kind_of_head) {
+    int nk = 0;
+    for (int h = 0; h < H; ++h) {
+        const int dl = dil ? dil[h] : 1;
+        int kidx = -1;
+        for (int a = 0; a < nk; ++a)
+            if (bp.dk_dil[a] == dl) kidx = a;
+        if (kidx < 0) {
+            kidx = nk++;
+            bp.dk_dil[kidx] = dl;
+            bp.dk_rows[kidx] = dl <= 4 ? 64 : 32;  // TMA box rows x stride <= 256
+        }
+        kind_of_head[h] = kidx;
+    }
+    for (int a = nk; a < kMaxDilKinds; ++a) {
+        bp.dk_dil[a] = 1;
+        bp.dk_rows[a] = 64;
+    }
+    return nk;
+}
+
+// The band kernel's work sequence and its split over at most max_ctas CTAs:
+// per (kind, class) and per head, block and tile offsets (band_tc.cuh).
+lf_status band_schedule(BandTcParams& bp, int B, int H, int T, int r_eff, int ngb, const int* kind_of_head,
+                        int max_ctas, long long tile_cap) {
+    bp.ngb = ngb;
+    for (int kd = 0; kd < kMaxDilKinds; ++kd) {
+        const int dl = bp.dk_dil[kd];
+        bp.dk_class_blk[kd][0] = 0;
+        bp.dk_class_tile[kd][0] = 0;
+        long long blk = 0, tiles = 0;
+        for (int c = 0; c < kMaxDilTma; ++c) {
+            if (c < dl) {
+                const int Tc = (T - c + dl - 1) / dl;
+                const int nt = (Tc + kBM - 1) / kBM;
+                for (int t = 0; t < nt; ++t) {
+                    int kbase = 0, kb_lo = 0, nbb = 0;
+                    tile_band(Tc, r_eff, t, kbase, kb_lo, nbb);
+                    blk += nbb + ngb;
+                }
+                tiles += nt;
+            }
+            if (blk > INT32_MAX) return LF_ERR_UNSUPPORTED;
+            bp.dk_class_blk[kd][c + 1] = static_cast<int>(blk);
+            bp.dk_class_tile[kd][c + 1] = static_cast<int>(tiles);
+        }
+    }
+    long long hb = 0, ht = 0;
+    for (int h = 0; h < H; ++h) {
+        const int kd = kind_of_head[h];
+        bp.head_blk[h] = static_cast<int>(hb);
+        bp.head_tile[h] = static_cast<int>(ht);
+        bp.head_dk[h] = static_cast<uint8_t>(kd);
+        hb += bp.dk_class_blk[kd][bp.dk_dil[kd]];
+        ht += bp.dk_class_tile[kd][bp.dk_dil[kd]];
+        if (hb > INT32_MAX) return LF_ERR_UNSUPPORTED;
+    }
+    for (int h = H; h <= kMaxHeads; ++h) {
+        bp.head_blk[h] = static_cast<int>(hb);
+        bp.head_tile[h] = static_cast<int>(ht);
+    }
+    bp.H = H;
+    bp.T = T;
+    bp.r = r_eff;
+    bp.blocks_per_b = static_cast<int>(hb);
+    bp.tiles_per_b = static_cast<int>(ht);
+    const long long nblk = static_cast<long long>(B) * hb;
+    if (nblk >= INT32_MAX || static_cast<long long>(B) * ht > tile_cap) return LF_ERR_UNSUPPORTED;
+    bp.n_blocks = static_cast<int>(nblk);
+    bp.grid_ctas = static_cast<int>(std::min<long long>(nblk, max_ctas));
+    bp.blk_q = bp.n_blocks / bp.grid_ctas;
+    bp.blk_rm = bp.n_blocks % bp.grid_ctas;
+    return LF_OK;
+}
+
 lf_status launch_all(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d, int r,
                      const int32_t* dil, const int32_t* gidx, int n_global, const uint8_t* pad, float scale,
                      lf_dtype dtype, cudaStream_t stream, DeviceState* ds, uint32_t stages = 7u) {
@@ -273,6 +362,8 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
     pp.ngp = L.ngp;
     pp.W = L.W;
     pp.pack = (dtype == LF_BF16 && n_global > 0) ? 1 : 0;
+    pp.band_cnt = reinterpret_cast<int32_t*>(base + L.off_bcnt);
+    pp.n_band_cnt = static_cast<int>(L.band_tiles * 8);
     const size_t prep_smem = size_t(L.W + 2 * kPrepThreads + L.gstride) * 4;
     if (stages & 1u) {
         prep_kernel<<<B * H, kPrepThreads, prep_smem, stream>>>(pp);
@@ -314,51 +405,34 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         if (st != LF_OK) return st;
         static thread_local BandTcParams bp;  // large (tensor maps); filled per call
         std::memset(&bp, 0, sizeof(bp));
-        int nk = 0;
         int kind_of_head[kMaxHeads];
-        for (int h = 0; h < H; ++h) {
-            const int dl = dil ? dil[h] : 1;
-            int kidx = -1;
-            for (int a = 0; a < nk; ++a)
-                if (bp.dk_dil[a] == dl) kidx = a;
-            if (kidx < 0) {
-                kidx = nk++;
-                bp.dk_dil[kidx] = dl;
-                bp.dk_rows[kidx] = dl <= 2 ? 128 : (dl <= 4 ? 64 : 32);
-                const uint32_t R = static_cast<uint32_t>(bp.dk_rows[kidx]);
-                if ((st = encode_rows_map(&bp.tm_q[kidx], q, T, uint64_t(B) * H, R, dl)) != LF_OK ||
-                    (st = encode_rows_map(&bp.tm_k[kidx], k, T, uint64_t(B) * H, R, dl)) != LF_OK ||
-                    (st = encode_rows_map(&bp.tm_v[kidx], v, T, uint64_t(B) * H, R, dl)) != LF_OK)
-                    return st;
-            }
-            kind_of_head[h] = kidx;
+        const int nk = assign_kinds(bp, H, dil, kind_of_head);
+        for (int kd = 0; kd < nk; ++kd) {
+            const int dl = bp.dk_dil[kd];
+            const uint32_t R = static_cast<uint32_t>(bp.dk_rows[kd]);
+            if ((st = encode_rows_map(&bp.tm_q[kd], q, T, uint64_t(B) * H, R, dl)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_k[kd], k, T, uint64_t(B) * H, R, dl)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_v[kd], v, T, uint64_t(B) * H, R, dl)) != LF_OK)
+                return st;
         }
         for (int a = nk; a < kMaxDilKinds; ++a) {  // unused slots: valid maps, never read
             bp.tm_q[a] = bp.tm_q[0];
             bp.tm_k[a] = bp.tm_k[0];
             bp.tm_v[a] = bp.tm_v[0];
-            bp.dk_dil[a] = 1;
-            bp.dk_rows[a] = 128;
         }
         if (n_global > 0) {
-            if ((st = encode_rows_map(&bp.tm_kg, ws.kg, L.ngp, uint64_t(B) * H, 128, 1)) != LF_OK ||
-                (st = encode_rows_map(&bp.tm_vg, ws.vg, L.ngp, uint64_t(B) * H, 128, 1)) != LF_OK)
+            if ((st = encode_rows_map(&bp.tm_kg, ws.kg, L.ngp, uint64_t(B) * H, kBN, 1)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_vg, ws.vg, L.ngp, uint64_t(B) * H, kBN, 1)) != LF_OK)
                 return st;
         } else {
             bp.tm_kg = bp.tm_k[0];
             bp.tm_vg = bp.tm_v[0];
         }
-        int items_per_b = 0;
-        for (int h = 0; h < H; ++h) {
-            bp.head_start[h] = items_per_b;
-            bp.head_dk[h] = static_cast<uint8_t>(kind_of_head[h]);
-            const int dl = bp.dk_dil[kind_of_head[h]];
-            for (int c = 0; c < dl; ++c) {
-                const int Tc = (T - c + dl - 1) / dl;
-                items_per_b += (Tc + kBM - 1) / kBM;
-            }
-        }
-        for (int h = H; h <= kMaxHeads; ++h) bp.head_start[h] = items_per_b;
+        if ((st = band_schedule(bp, B, H, T, r_eff, n_global > 0 ? (L.gstride + kBN - 1) / kBN : 0, kind_of_head,
+                                std::min(kBandCtasPerSm * ds->sm_count, kMaxBandCtas), L.band_tiles)) != LF_OK)
+            return st;
+        bp.cnt = reinterpret_cast<int32_t*>(base + L.off_bcnt);
+        bp.part = reinterpret_cast<float*>(base + L.off_bpart);
         bp.out = static_cast<__nv_bfloat16*>(out);
         bp.pad = pad;
         bp.gk_list = ws.gk_list;
@@ -369,49 +443,10 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         bp.W = L.W;
         bp.gstride = L.gstride;
         bp.sl2 = sl2;
-        bp.items_per_b = items_per_b;
-        bp.n_items = items_per_b * B;
-        bp.item_order = nullptr;
-        if (ds->may_order) {
-            // Longest tiles first: with fewer CTAs than tiles, the CTAs that take a second
-            // tile then take one of the short tiles at the sequence ends.
-            std::vector<int> key = {B, H, T, r_eff};
-            for (int h = 0; h < H; ++h) key.push_back(dil ? dil[h] : 1);
-            if (key != ds->order_key && !is_capturing(stream)) {
-                std::vector<int> cost;
-                cost.reserve(bp.n_items);
-                for (int b = 0; b < B; ++b)
-                    for (int h = 0; h < H; ++h) {
-                        const int dl = bp.dk_dil[kind_of_head[h]];
-                        for (int c = 0; c < dl; ++c) {
-                            const int Tc = (T - c + dl - 1) / dl;
-                            for (int q0 = 0; q0 < Tc; q0 += kBM) {
-                                const int kbase = q0 - r_eff;
-                                const int lo = std::max(0, kbase), hi = std::min(Tc - 1, q0 + kBM - 1 + r_eff);
-                                cost.push_back((hi - kbase) / kBN + 1 - (lo - kbase) / kBN);
-                            }
-                        }
-                    }
-                std::vector<int32_t> order(cost.size());
-                for (size_t a = 0; a < order.size(); ++a) order[a] = static_cast<int32_t>(a);
-                std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) { return cost[x] > cost[y]; });
-                bool identity = true;
-                for (size_t a = 0; a < order.size() && identity; ++a) identity = order[a] == static_cast<int32_t>(a);
-                if (!identity) {
-                    void* buf = ds->order;
-                    if ((st = grow(&buf, &ds->order_cap, order.size() * sizeof(int32_t), stream)) != LF_OK) return st;
-                    ds->order = static_cast<int32_t*>(buf);
-                    // from pageable memory: returns once the data is staged, ordered on the stream
-                    if (cudaMemcpyAsync(ds->order, order.data(), order.size() * sizeof(int32_t),
-                                        cudaMemcpyHostToDevice, stream) != cudaSuccess)
-                        return LF_ERR_CUDA;
-                }
-                ds->order_identity = identity;
-                ds->order_key = key;
-            }
-            if (key == ds->order_key && !ds->order_identity) bp.item_order = ds->order;
-        }
-        const int grid = std::min(bp.n_items, kBandCtasPerSm * ds->sm_count);
+        const unsigned long long wl = g_test_wait_ns.load();
+        bp.wait_ns = wl ? wl : LF_WAIT_NS;
+        bp.test_stall = g_test_stall.load();
+        const int grid = bp.grid_ctas;  // persistent: two CTAs per SM
         // right after prep on the same stream, launched as its programmatic dependent: the
         // band kernel's set-up (barriers, TMEM, tensor-map prefetch) overlaps prep
         cudaLaunchConfig_t cfg = {};
@@ -581,8 +616,6 @@ lf_status lf_attn_fwd_host(const void* q, const void* k, const void* v, void* ou
     const bool sliced = nslices > 1 && nslices <= DeviceState::kMaxSlices;
     const int slice_h = sliced ? hg : H;
     const size_t per_head = size_t(T) * d * es;
-    const bool saved_order = ds->may_order;
-    ds->may_order = !sliced;  // one tile order per call: the slices would keep rebuilding it
     int a = 0;
     for (int b = 0; b < (sliced ? B : 1) && st == LF_OK; ++b)
         for (int h0 = 0; h0 < H && st == LF_OK; h0 += slice_h, ++a) {
@@ -611,7 +644,6 @@ lf_status lf_attn_fwd_host(const void* q, const void* k, const void* v, void* ou
                                 ds->cout) != cudaSuccess)
                 st = LF_ERR_CUDA;
         }
-    ds->may_order = saved_order;
     // everything queued so far must finish before the staging area is reused or `out` is read
     const bool synced = cudaStreamSynchronize(ds->cin) == cudaSuccess &&
                         cudaStreamSynchronize(s) == cudaSuccess && cudaStreamSynchronize(ds->cout) == cudaSuccess;
@@ -658,7 +690,6 @@ void lf_attn_release(void) {
         cudaSetDevice(dev);
         if (s.ws) cudaFree(s.ws);
         if (s.io) cudaFree(s.io);
-        if (s.order) cudaFree(s.order);
         if (s.status) cudaFree(s.status);
         if (s.ev_fork) cudaEventDestroy(s.ev_fork);
         if (s.ev_join) cudaEventDestroy(s.ev_join);
@@ -681,6 +712,58 @@ uint64_t lf_attn_workspace_bytes(int B, int H, int T, int d, int n_global, lf_dt
 
 int lf_attn_last_launch_count(void) { return t_last_launches; }
 
+void lf_attn_test_hooks(uint32_t flags, uint64_t wait_ns) {
+    g_test_stall.store((flags & 1u) ? 1 : 0);
+    g_test_wait_ns.store(wait_ns);
+}
+
+int lf_attn_band_plan(int B, int H, int T, int r, const int32_t* dil, int n_global, int max_ctas, int32_t* pieces,
+                      int capacity) {
+    if (B <= 0 || H <= 0 || H > kMaxHeads || T <= 0 || r < 0 || n_global < 0 || max_ctas <= 0) return -1;
+    for (int h = 0; h < H; ++h)
+        if (dil && (dil[h] < 1 || dil[h] > kMaxDilTma)) return -1;
+    static thread_local BandTcParams bp;
+    std::memset(&bp, 0, sizeof(bp));
+    int kind_of_head[kMaxHeads];
+    if (assign_kinds(bp, H, dil, kind_of_head) > kMaxDilKinds) return -1;
+    const int r_eff = std::min(r, T);
+    const int gstride = std::max(1, std::min(n_global, T));
+    const Layout L = make_layout(B, H, T, 64, n_global, LF_BF16);
+    if (band_schedule(bp, B, H, T, r_eff, n_global > 0 ? (gstride + kBN - 1) / kBN : 0, kind_of_head,
+                      std::min(max_ctas, kMaxBandCtas), L.band_tiles) != LF_OK)
+        return -1;
+    bp.B = B;
+    // the walk each CTA's producer makes (band_tc.cuh), on the host
+    int n = 0;
+    for (int s = 0; s < bp.grid_ctas; ++s) {
+        const int x0 = range_start(bp, s), x1 = range_start(bp, s + 1);
+        TileWalker w;
+        w.locate(bp, x0);
+        for (int x = x0; x < x1;) {
+            const int tend = w.start + w.nb(bp);
+            const int pend = std::min(tend, x1);
+            if (pieces && n < capacity) {
+                int32_t* e = pieces + size_t(n) * 10;
+                e[0] = s;
+                e[1] = w.tile;
+                e[2] = static_cast<int32_t>(x - w.start);
+                e[3] = static_cast<int32_t>(pend - w.start);
+                e[4] = w.nb(bp);
+                e[5] = cta_of(bp, w.start);
+                e[6] = cta_of(bp, tend - 1);
+                e[7] = 2 * s + (w.start > x0 ? 1 : 0);  // partial slot (band_tc.cuh part_slot)
+                e[8] = w.b * H + w.h;
+                e[9] = w.c * 65536 + w.t;
+            }
+            ++n;
+            x = pend;
+            if (x < x1) w.next(bp);
+        }
+    }
+    return n;
+}
+
+
 lf_status lf_attn_fwd_static(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d,
                              int r, const int32_t* dil, const int32_t* global_idx, int n_global,
                              const uint8_t* key_pad_mask, float scale, lf_dtype dtype, void* stream) {
@@ -695,7 +778,6 @@ lf_status lf_attn_fwd_static(const void* q, const void* k, const void* v, void* 
     // never grows (allocates) it.  Prep zeroes what must start at zero.
     DeviceState view;
     view.init = true;
-    view.may_order = false;
     view.sm_count = ss->sm_count;
     view.status = reinterpret_cast<uint32_t*>(ss->scratch);
     view.ws = ss->scratch + 256;

@@ -33,6 +33,8 @@ struct Workspace {
 
 struct PrepParams {
     const int32_t* gidx;  // [B][n_global] or null
+    int32_t* band_cnt;    // band kernel merge tickets, zeroed here (n_band_cnt entries)
+    int n_band_cnt;
     const uint8_t* pad;   // [B][T] or null
     const void* k;        // [B,H,T,d] (bf16 path: packed into kg)
     const void* v;
@@ -78,15 +80,26 @@ struct BandTcParams {
     const int32_t* n_gk;
     const uint32_t* gbit;
     uint32_t* status;
+    int32_t* cnt;  // [tiles][4][2] merge tickets and lanes done writing (zero between calls)
+    float* part;   // [2 * grid_ctas] partial states of split tiles
     int B, H, T, r, W, gstride;
     float sl2;
-    int n_items;     // work items (b, h, residue class, 128-query tile)
-    int items_per_b;
+    unsigned long long wait_ns;  // limit of every pipeline wait (drains keep their own)
+    int test_stall;              // test hook: the producers publish nothing
+    // The work sequence: per sample, heads in order; per head, residue
+    // classes; per class, 128-query tiles; per tile, nbb band blocks then ngb
+    // global blocks.  CTA s takes blocks [s*N/G, (s+1)*N/G).
+    int n_blocks;        // N (< 2^31)
+    int grid_ctas;       // G
+    int blk_q, blk_rm;   // N = blk_q * G + blk_rm
+    int blocks_per_b, tiles_per_b, ngb;
     int dk_dil[kMaxDilKinds];
-    int dk_rows[kMaxDilKinds];   // rows per TMA box for that dilation
-    int head_start[kMaxHeads + 1];  // item offset of each head inside one sample
+    int dk_rows[kMaxDilKinds];                          // rows per TMA box for that dilation
+    int dk_class_blk[kMaxDilKinds][kMaxDilTma + 1];     // block offset of class c in a head of that kind
+    int dk_class_tile[kMaxDilKinds][kMaxDilTma + 1];    // tile offset of class c
+    int head_blk[kMaxHeads + 1];                        // block offset of head h in a sample
+    int head_tile[kMaxHeads + 1];                       // tile offset of head h in a sample
     uint8_t head_dk[kMaxHeads];
-    const int32_t* item_order;  // work slot -> item (longest tiles first); null: slot = item
 };
 
 }  // namespace lf

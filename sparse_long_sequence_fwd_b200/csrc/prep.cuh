@@ -10,7 +10,8 @@
 // is removed as a key ("Implementation Reading": padding must be masked) but
 // is still a global query.  Entries outside [0, T) are ignored and raise the
 // status bit.  It also zeroes the arrival counters the global-row kernel
-// uses for its (b, h).  On the bf16 path every CTA also packs the rows of k and v
+// uses for its (b, h), and (all CTAs together) the band kernel's merge
+// tickets.  On the bf16 path every CTA also packs the rows of k and v
 // named by gk_list into contiguous [ngp][64] blocks for its (b, h), zero
 // beyond the list, so the band kernel can stage them with one TMA box.
 #pragma once
@@ -63,6 +64,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
 
     for (int w = tid; w < p.W; w += kPrepThreads) bits[w] = 0u;
     if (tid == 0) p.ws.counters[blockIdx.x] = 0;  // arrival tickets of the global-row kernel
+    for (int a = blockIdx.x * kPrepThreads + tid; a < p.n_band_cnt; a += gridDim.x * kPrepThreads)
+        p.band_cnt[a] = 0;  // the band kernel's merge tickets (its mergers also reset what they use)
     __syncthreads();
     for (int a = tid; a < p.n_global; a += kPrepThreads) {
         int g = p.gidx[static_cast<size_t>(b) * p.n_global + a];

@@ -20,7 +20,7 @@ STATUS = {0: "LF_OK", 1: "LF_ERR_INVALID_ARG", 2: "LF_ERR_UNSUPPORTED", 3: "LF_E
           4: "LF_ERR_NO_MEMORY", 5: "LF_ERR_DEVICE_CHECK", 6: "LF_ERR_SCRATCH_TOO_SMALL"}
 EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
            "lf_attn_release", "lf_attn_workspace_bytes", "lf_attn_last_launch_count",
-           "lf_attn_fwd_static")
+           "lf_attn_fwd_static", "lf_attn_band_plan", "lf_attn_test_hooks")
 
 _lib = None
 
@@ -58,6 +58,10 @@ def load():
         lib.lf_attn_last_launch_count.restype = I
         lib.lf_attn_fwd_static.argtypes = sig
         lib.lf_attn_fwd_static.restype = I
+        lib.lf_attn_band_plan.argtypes = [I, I, I, I, P, I, I, P, I]
+        lib.lf_attn_band_plan.restype = I
+        lib.lf_attn_test_hooks.argtypes = [ctypes.c_uint32, ctypes.c_uint64]
+        lib.lf_attn_test_hooks.restype = None
 
         _lib = lib
     return _lib
@@ -205,6 +209,28 @@ def workspace_bytes(B, H, T, d, n_global, dtype_code) -> int:
 
 def last_launch_count() -> int:
     return int(load().lf_attn_last_launch_count())
+
+
+def band_plan(B: int, H: int, T: int, r: int, dil=None, n_global: int = 0, max_ctas: int = 296):
+    """The band kernel's split of its work over at most ``max_ctas`` pipelines
+    (computed on the host, no device needed): an int32 array [pieces, 10] of
+    (pipeline, tile, first block, end block, blocks of the tile, first and
+    last pipeline of the tile, partial-state slot, b*H + h, class*65536 + t)."""
+    import numpy as np
+    d = _dil_array(dil, H)
+    n = load().lf_attn_band_plan(B, H, T, int(r), d, int(n_global), int(max_ctas), None, 0)
+    if n < 0:
+        raise ValueError("lf_attn_band_plan rejected these sizes")
+    out = np.zeros((max(n, 1), 10), dtype=np.int32)
+    m = load().lf_attn_band_plan(B, H, T, int(r), d, int(n_global), int(max_ctas),
+                                 ctypes.c_void_p(out.ctypes.data), n)
+    assert m == n
+    return out[:n]
+
+
+def test_hooks(flags: int = 0, wait_ns: int = 0) -> None:
+    """Test hook of the band kernel's failure path (see lf_attn_test_hooks)."""
+    load().lf_attn_test_hooks(int(flags), int(wait_ns))
 
 
 def raw_call(name: str, *args) -> int:
