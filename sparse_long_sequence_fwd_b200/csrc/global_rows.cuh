@@ -190,20 +190,27 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
 
 // bf16, d = 64: tensor-core global rows.  CTA (split, b*h, row group) takes
 // up to 64 global queries of sample b (16 per warp: one m16n8k16 row tile)
-// and cpc consecutive 128-key chunks of the key axis.  Each chunk of K and V
-// is staged once in padded shared memory (cp.async, zero-filled past T);
-// every warp forms S = Q K^T (16 x 128, fp32 in registers), applies the key
-// padding mask, runs the online softmax (log2 domain, exp2) and accumulates
-// O += P V with P re-packed from the S registers as bf16 A fragments and V
-// fragments from ldmatrix.trans.  The partial state (m, l, O) of each row and
-// split goes to the workspace; global_rows_merge_kernel combines the splits.
-// This path is bound by HBM traffic (every K/V row of a (b, h) is read once
-// per row group), not by the tensor rate, so the synchronous warp-level MMA
-// is enough.
+// and cpc consecutive 128-key chunks of the key axis.  The chunks of K and V
+// stream through a two-stage ring in padded shared memory (cp.async,
+// zero-filled past T); the first two are requested before anything that
+// depends on the prep kernel (the global-query count and list, the query
+// rows), so the HBM latency overlaps those reads.  Every warp forms
+// S = Q K^T (16 x 128, fp32 in registers), applies the key padding mask,
+// runs the online softmax (log2 domain, exp2) and accumulates O += P V with
+// P re-packed from the S registers as bf16 A fragments and V fragments from
+// ldmatrix.trans.  The partial state (m, l, O) of each row and split goes to
+// the workspace; global_rows_merge_kernel combines the splits.  This path is
+// bound by HBM traffic (every K/V row of a (b, h) is read once per row
+// group), not by the tensor rate, so the synchronous warp-level MMA is
+// enough.
 constexpr int kGrKeys = 128;       // keys per chunk
 constexpr int kGrWarps = 4;        // 16 rows per warp
 constexpr int kGrRows = 16 * kGrWarps;
 constexpr int kGrStride = 72;      // bf16 per staged row: 64 + 8 (conflict-free fragments and ldmatrix)
+constexpr int kGrStages = 2;
+constexpr int kGrChunkElems = kGrKeys * kGrStride;          // bf16 per K (or V) chunk
+constexpr int kGrSmem = kGrStages * 2 * kGrChunkElems * 2;  // bytes of the ring
+constexpr int kMaxSplits = 64;                              // key splits per (b, h): the merge holds them in registers
 
 __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -227,22 +234,45 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__global__ void __launch_bounds__(kGrWarps * 32) global_rows_mma_kernel(const __grid_constant__ GlobalRowParams p) {
-    __shared__ __align__(16) __nv_bfloat16 Ks[kGrKeys * kGrStride];
-    __shared__ __align__(16) __nv_bfloat16 Vs[kGrKeys * kGrStride];
-    __shared__ uint32_t valid_bits[kGrKeys / 32];
+__global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const __grid_constant__ GlobalRowParams p) {
+    extern __shared__ __align__(16) __nv_bfloat16 gr_ring[];  // [stage][K, V][kGrKeys][kGrStride]
+    __shared__ uint32_t valid_bits[kGrStages][kGrKeys / 32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g8 = lane >> 2, t4 = lane & 3;  // fragment row group and column pair
     const int split = blockIdx.x, bh = blockIdx.y, b = bh / p.H;
-    const int nq = p.ws.n_gq[b];
-    const int row0 = blockIdx.z * kGrRows + warp * 16;  // this warp's first global-row slot
-    if (blockIdx.z * kGrRows >= nq) return;
     const int T = p.T;
     const size_t base = static_cast<size_t>(bh) * T * 64;
     const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(p.k) + base;
     const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(p.v) + base;
     const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(p.q) + base;
+    const int nblk = (T + kGrKeys - 1) / kGrKeys;
+    const int c_lo = split * p.cpc, c_hi = min(nblk, c_lo + p.cpc);
+
+    // one commit group per chunk: its K and V into ring stage st
+    auto issue = [&](int ch, int st) {
+        const int j0 = ch * kGrKeys;
+        __nv_bfloat16* Ks = gr_ring + st * 2 * kGrChunkElems;
+        __nv_bfloat16* Vs = Ks + kGrChunkElems;
+        for (int u = tid; u < kGrKeys * 8; u += kGrWarps * 32) {
+            const int key = u >> 3, part = u & 7;
+            const bool in = j0 + key < T;
+            const size_t src = static_cast<size_t>(in ? j0 + key : 0) * 64 + part * 8;
+            cp_async16(Ks + key * kGrStride + part * 8, kb + src, in ? 16u : 0u);
+            cp_async16(Vs + key * kGrStride + part * 8, vb + src, in ? 16u : 0u);
+        }
+    };
+    issue(c_lo, 0);
+    cp_async_commit();
+    if (c_lo + 1 < c_hi) issue(c_lo + 1, 1);
+    cp_async_commit();
+
+    const int nq = p.ws.n_gq[b];
+    const int row0 = blockIdx.z * kGrRows + warp * 16;  // this warp's first global-row slot
+    if (blockIdx.z * kGrRows >= nq) {
+        cp_async_wait<0>();  // no copy may still target this CTA's shared memory
+        return;
+    }
     const int32_t* gq = p.ws.gq_list + static_cast<size_t>(b) * p.gstride;
     const bool active = row0 < nq;
 
@@ -267,115 +297,99 @@ __global__ void __launch_bounds__(kGrWarps * 32) global_rows_mma_kernel(const __
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;  // rows g8, g8 + 8
     const float sl2 = p.sl2;
 
-    const int nblk = (T + kGrKeys - 1) / kGrKeys;
-    const int c_lo = split * p.cpc, c_hi = min(nblk, c_lo + p.cpc);
     for (int ch = c_lo; ch < c_hi; ++ch) {
-        const int j0 = ch * kGrKeys;
-        __syncthreads();  // previous chunk fully consumed
-        // K, then V, as two groups: S and the softmax run while V is still arriving
-        for (int u = tid; u < kGrKeys * 8; u += kGrWarps * 32) {
-            const int key = u >> 3, part = u & 7;
-            const bool in = j0 + key < T;
-            const size_t src = static_cast<size_t>(in ? j0 + key : 0) * 64 + part * 8;
-            cp_async16(Ks + key * kGrStride + part * 8, kb + src, in ? 16u : 0u);
-        }
-        cp_async_commit();
-        for (int u = tid; u < kGrKeys * 8; u += kGrWarps * 32) {
-            const int key = u >> 3, part = u & 7;
-            const bool in = j0 + key < T;
-            const size_t src = static_cast<size_t>(in ? j0 + key : 0) * 64 + part * 8;
-            cp_async16(Vs + key * kGrStride + part * 8, vb + src, in ? 16u : 0u);
-        }
-        cp_async_commit();
-        if (tid < kGrKeys) {
-            const int j = j0 + tid;
+        const int st = (ch - c_lo) & 1;
+        const __nv_bfloat16* Ks = gr_ring + st * 2 * kGrChunkElems;
+        const __nv_bfloat16* Vs = Ks + kGrChunkElems;
+        if (tid < kGrKeys) {  // valid keys of this chunk (inside T, not padded)
+            const int j = ch * kGrKeys + tid;
             const bool ok = j < T && !(p.pad && p.pad[static_cast<size_t>(b) * T + j]);
             const uint32_t w = __ballot_sync(0xffffffffu, ok);
-            if (lane == 0) valid_bits[tid >> 5] = w;
+            if (lane == 0) valid_bits[st][tid >> 5] = w;
         }
-        cp_async_wait<1>();  // K has landed
+        cp_async_wait<1>();  // this chunk has landed (the next one may still be in flight)
         __syncthreads();
-        uint32_t pa[8][4];  // P of this warp's rows as bf16 A fragments
         if (active) {
-
-        // S = Q K^T: 16 key tiles of 8
-        float s[16][4];
+            // S = Q K^T: 16 key tiles of 8
+            float s[16][4];
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-            const __nv_bfloat16* kr = Ks + (8 * nt + g8) * kGrStride + 2 * t4;
+            for (int nt = 0; nt < 16; ++nt) {
+                s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+                const __nv_bfloat16* kr = Ks + (8 * nt + g8) * kGrStride + 2 * t4;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks);
-                const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks + 8);
-                mma_bf16_16816(s[nt], qa[ks], b0, b1);
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks);
+                    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks + 8);
+                    mma_bf16_16816(s[nt], qa[ks], b0, b1);
+                }
+            }
+            // mask, scale, row maxima (each row's 128 scores live in the 4 lanes of its quad)
+            float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                const uint32_t vw = valid_bits[st][nt >> 2] >> ((nt & 3) * 8 + 2 * t4);
+                const bool v0 = vw & 1u, v1 = (vw >> 1) & 1u;
+                s[nt][0] = v0 ? s[nt][0] * sl2 : -INFINITY;
+                s[nt][1] = v1 ? s[nt][1] * sl2 : -INFINITY;
+                s[nt][2] = v0 ? s[nt][2] * sl2 : -INFINITY;
+                s[nt][3] = v1 ? s[nt][3] * sl2 : -INFINITY;
+                mx_a = fmaxf(mx_a, fmaxf(s[nt][0], s[nt][1]));
+                mx_b = fmaxf(mx_b, fmaxf(s[nt][2], s[nt][3]));
+            }
+#pragma unroll
+            for (int off = 1; off <= 2; off <<= 1) {
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+            }
+            const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+            const float al_a = m_a == -INFINITY ? 0.f : exp2f(m_a - mn_a);
+            const float al_b = m_b == -INFINITY ? 0.f : exp2f(m_b - mn_b);
+            m_a = mn_a;
+            m_b = mn_b;
+            const float bs_a = mn_a == -INFINITY ? 0.f : mn_a, bs_b = mn_b == -INFINITY ? 0.f : mn_b;
+            l_a *= al_a;
+            l_b *= al_b;
+#pragma unroll
+            for (int nd = 0; nd < 8; ++nd) {
+                o[nd][0] *= al_a;
+                o[nd][1] *= al_a;
+                o[nd][2] *= al_b;
+                o[nd][3] *= al_b;
+            }
+            // P (bf16 A fragments) and row sums
+            uint32_t pa[8][4];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float* sv = s[2 * kk + h];
+                    const float e0 = exp2f(sv[0] - bs_a), e1 = exp2f(sv[1] - bs_a);
+                    const float e2 = exp2f(sv[2] - bs_b), e3 = exp2f(sv[3] - bs_b);
+                    l_a += e0 + e1;
+                    l_b += e2 + e3;
+                    pa[kk][2 * h] = pack_bf16x2(e0, e1);
+                    pa[kk][2 * h + 1] = pack_bf16x2(e2, e3);
+                }
+            }
+            // O += P V: for each 16-key step, two 8-column tiles of V per ldmatrix
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t a4[4] = {pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3]};
+#pragma unroll
+                for (int nd = 0; nd < 8; nd += 2) {
+                    uint32_t vf[4];
+                    ldmatrix_x4_trans(vf, Vs + (16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1)) * kGrStride +
+                                              8 * (nd + (lane >> 4)));
+                    mma_bf16_16816(o[nd], a4, vf[0], vf[1]);
+                    mma_bf16_16816(o[nd + 1], a4, vf[2], vf[3]);
+                }
             }
         }
-        // mask, scale, row maxima (each row's 128 scores live in the 4 lanes of its quad)
-        float mx_a = -INFINITY, mx_b = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const uint32_t vw = valid_bits[nt >> 2] >> ((nt & 3) * 8 + 2 * t4);
-            const bool v0 = vw & 1u, v1 = (vw >> 1) & 1u;
-            s[nt][0] = v0 ? s[nt][0] * sl2 : -INFINITY;
-            s[nt][1] = v1 ? s[nt][1] * sl2 : -INFINITY;
-            s[nt][2] = v0 ? s[nt][2] * sl2 : -INFINITY;
-            s[nt][3] = v1 ? s[nt][3] * sl2 : -INFINITY;
-            mx_a = fmaxf(mx_a, fmaxf(s[nt][0], s[nt][1]));
-            mx_b = fmaxf(mx_b, fmaxf(s[nt][2], s[nt][3]));
-        }
-#pragma unroll
-        for (int off = 1; off <= 2; off <<= 1) {
-            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
-            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
-        }
-        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-        const float al_a = m_a == -INFINITY ? 0.f : exp2f(m_a - mn_a);
-        const float al_b = m_b == -INFINITY ? 0.f : exp2f(m_b - mn_b);
-        m_a = mn_a;
-        m_b = mn_b;
-        const float bs_a = mn_a == -INFINITY ? 0.f : mn_a, bs_b = mn_b == -INFINITY ? 0.f : mn_b;
-        l_a *= al_a;
-        l_b *= al_b;
-#pragma unroll
-        for (int nd = 0; nd < 8; ++nd) {
-            o[nd][0] *= al_a;
-            o[nd][1] *= al_a;
-            o[nd][2] *= al_b;
-            o[nd][3] *= al_b;
-        }
-        // P (bf16 A fragments) and row sums
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float* sv = s[2 * kk + h];
-                const float e0 = exp2f(sv[0] - bs_a), e1 = exp2f(sv[1] - bs_a);
-                const float e2 = exp2f(sv[2] - bs_b), e3 = exp2f(sv[3] - bs_b);
-                l_a += e0 + e1;
-                l_b += e2 + e3;
-                pa[kk][2 * h] = pack_bf16x2(e0, e1);
-                pa[kk][2 * h + 1] = pack_bf16x2(e2, e3);
-            }
-        }
-        }
-        cp_async_wait<0>();  // V has landed
-        __syncthreads();
-        if (!active) continue;
-        // O += P V: for each 16-key step, two 8-column tiles of V per ldmatrix
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a[4] = {pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3]};
-#pragma unroll
-            for (int nd = 0; nd < 8; nd += 2) {
-                uint32_t vf[4];
-                ldmatrix_x4_trans(vf, Vs + (16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1)) * kGrStride +
-                                          8 * (nd + (lane >> 4)));
-                mma_bf16_16816(o[nd], a, vf[0], vf[1]);
-                mma_bf16_16816(o[nd + 1], a, vf[2], vf[3]);
-            }
-        }
+        __syncthreads();  // this stage is consumed: the chunk two ahead may overwrite it
+        if (ch + 2 < c_hi) issue(ch + 2, st);
+        cp_async_commit();  // (empty past the last chunk, so every wait above counts the same)
     }
+    cp_async_wait<0>();
     if (!active) return;
     // full row sums over the quad, then the partial state of each row
 #pragma unroll
@@ -404,51 +418,53 @@ __global__ void __launch_bounds__(kGrWarps * 32) global_rows_mma_kernel(const __
 
 // One CTA per (global-row slot, b*h), one thread per output column: the
 // splits' partial states combine as M = max_c m_c, w_c = 2^(m_c - M),
-// y = sum_c w_c acc_c / sum_c w_c l_c.  The maxima and weights are formed
-// cooperatively (strided over the splits), then every thread streams its
-// column of the partial accumulators with independent loads.
-constexpr int kMaxSplits = 1024;  // the host keeps the split count near 600 CTAs' worth
+// y = sum_c w_c acc_c / sum_c w_c l_c.  Launched as the split kernel's
+// programmatic dependent (its launch overlaps the splits' end).  Every load
+// of a pass is issued before any of its values is used, so each pass costs
+// one round trip to L2.
 __global__ void __launch_bounds__(64) global_rows_merge_kernel(const __grid_constant__ GlobalRowParams p) {
     __shared__ float wsh[kMaxSplits];
     __shared__ float red[2];
+    grid_dep_wait();  // the split kernel's partial states are complete and visible
     const int a = blockIdx.x, bh = blockIdx.y, b = bh / p.H;
     if (a >= p.ws.n_gq[b]) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nsplit = p.nchunk;
     const float* src = p.ws.partial + (static_cast<size_t>(bh) * p.gstride + a) * nsplit * 66;
+    const int32_t g = p.ws.gq_list[static_cast<size_t>(b) * p.gstride + a];
 
-    float M = -INFINITY;
-    for (int c = tid; c < nsplit; c += 64) M = fmaxf(M, __ldcg(src + static_cast<size_t>(c) * 66));
+    // pass 1: every split's (m, l); thread c holds split c (nsplit <= 64)
+    const float mc = tid < nsplit ? __ldcg(src + static_cast<size_t>(tid) * 66) : -INFINITY;
+    const float lc = tid < nsplit ? __ldcg(src + static_cast<size_t>(tid) * 66 + 1) : 0.f;
+    float M = mc;
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     if (lane == 0) red[warp] = M;
     __syncthreads();
     M = fmaxf(red[0], red[1]);
     const float Mu = M == -INFINITY ? 0.f : M;  // every split empty: all weights 0
-    __syncthreads();
-    float L = 0.f;
-    for (int c = tid; c < nsplit; c += 64) {
-        const float* q = src + static_cast<size_t>(c) * 66;
-        const float w = exp2f(__ldcg(q) - Mu);  // m_c = -inf gives 0
-        wsh[c] = w;
-        L = fmaf(w, __ldcg(q + 1), L);
-    }
+    const float wc = exp2f(mc - Mu);            // m = -inf gives 0
+    if (tid < nsplit) wsh[tid] = wc;
+    float L = wc * lc;
 #pragma unroll
     for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    __syncthreads();
     if (lane == 0) red[warp] = L;
     __syncthreads();
     L = red[0] + red[1];
-    float acc0 = 0.f, acc1 = 0.f;
+
+    // pass 2: column tid of every split, all loads first
+    float v[kMaxSplits];
     const float* col = src + 2 + tid;
-    int c = 0;
-#pragma unroll 4
-    for (; c + 1 < nsplit; c += 2) {
-        acc0 = fmaf(wsh[c], __ldcg(col + static_cast<size_t>(c) * 66), acc0);
-        acc1 = fmaf(wsh[c + 1], __ldcg(col + static_cast<size_t>(c + 1) * 66), acc1);
+#pragma unroll
+    for (int c = 0; c < kMaxSplits; ++c) v[c] = c < nsplit ? __ldcg(col + static_cast<size_t>(c) * 66) : 0.f;
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxSplits; c += 2) {
+        if (c < nsplit) acc0 = fmaf(wsh[c], v[c], acc0);
+        if (c + 1 < nsplit) acc1 = fmaf(wsh[c + 1], v[c + 1], acc1);
     }
-    if (c < nsplit) acc0 = fmaf(wsh[c], __ldcg(col + static_cast<size_t>(c) * 66), acc0);
     const float y = L > 0.f ? (acc0 + acc1) / L : 0.f;
-    const int32_t g = p.ws.gq_list[static_cast<size_t>(b) * p.gstride + a];
     reinterpret_cast<__nv_bfloat16*>(p.out)[(static_cast<size_t>(bh) * p.T + g) * 64 + tid] = __float2bfloat16_rn(y);
 }
 

@@ -76,10 +76,11 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
     L.W = (T + 31) / 32;
     L.gstride = std::max(1, std::min(n_global, T));
     if (dtype == LF_BF16) {
-        // tensor-core global rows: 128-key chunks, cpc per CTA, about 600 CTAs in all
+        // tensor-core global rows: 128-key chunks, cpc per CTA, about three CTAs
+        // per SM of a 148-SM B200 (each holds a two-stage ring of 72 KB)
         const int nblk = (T + kGrKeys - 1) / kGrKeys;
         const long units = long(nblk) * B * H * ((L.gstride + kGrRows - 1) / kGrRows);
-        L.cpc = static_cast<int>(std::max(1L, std::min<long>(nblk, units / 600)));
+        L.cpc = static_cast<int>(std::max(1L, std::min<long>(nblk, (units + 443) / 444)));
         L.nchunk = (nblk + L.cpc - 1) / L.cpc;
         while (L.nchunk > kMaxSplits) L.nchunk = (nblk + ++L.cpc - 1) / L.cpc;
     } else {
@@ -136,7 +137,8 @@ lf_status set_kernel_attributes() {
         cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
             cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
-            cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) != cudaSuccess)
         return LF_ERR_CUDA;
     return LF_OK;
 }
@@ -484,9 +486,20 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         gp.cpc = L.cpc;
         if (dtype == LF_BF16) {
             // key splits x (b, h) x groups of 64 global rows, then the merge of the splits
-            global_rows_mma_kernel<<<dim3(L.nchunk, B * H, (L.gstride + kGrRows - 1) / kGrRows), kGrWarps * 32, 0,
-                                     gs>>>(gp);
-            global_rows_merge_kernel<<<dim3(L.gstride, B * H), 64, 0, gs>>>(gp);
+            global_rows_mma_kernel<<<dim3(L.nchunk, B * H, (L.gstride + kGrRows - 1) / kGrRows), kGrWarps * 32,
+                                     kGrSmem, gs>>>(gp);
+            // the merge is the split kernel's programmatic dependent: it launches while the
+            // splits finish and waits for them (griddepcontrol.wait) before reading
+            cudaLaunchConfig_t mc = {};
+            mc.gridDim = dim3(static_cast<unsigned>(L.gstride), static_cast<unsigned>(B * H));
+            mc.blockDim = dim3(64);
+            mc.stream = gs;
+            cudaLaunchAttribute mattr[1];
+            mattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            mattr[0].val.programmaticStreamSerializationAllowed = 1;
+            mc.attrs = mattr;
+            mc.numAttrs = 1;
+            if (cudaLaunchKernelEx(&mc, global_rows_merge_kernel, gp) != cudaSuccess) return LF_ERR_CUDA;
             launches += 2;
         } else {
             const dim3 grid(L.nchunk, B * H);
