@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-others", action="store_true", help="skip the QA, dilated and large workload entries")
     return ap.parse_args()
 
 
@@ -192,6 +193,123 @@ def traffic_from_profile(kernel_file: str):
 
 
 # ---------------------------------------------------------------------------- ours
+class WorkloadRun:
+    """One workload on one GPU: rotating input sets (together more than twice
+    the L2 size, so every step reads q/k/v from DRAM), CUDA graphs of steps
+    and of single stages, timed with CUDA events on the launching stream."""
+
+    def __init__(self, w, torch, lf_attn, dev, stream, warmup):
+        self.w, self.torch, self.lf_attn, self.stream = w, torch, lf_attn, stream
+        self.inp = inp = workloads.make_inputs(w)
+        self.total_f, self.band_f, self.gr_f, self.gr_bytes = split_flops(w, inp)
+        props = torch.cuda.get_device_properties(dev)
+        self.l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
+        es = 2 if w.dtype == "bf16" else 4
+        self.set_bytes = 4 * w.B * w.H * w.T * w.d * es
+        self.n_sets = max(2, math.ceil(2 * self.l2 / self.set_bytes) + 1)
+        q0, k0, v0 = (inp[x].to(dev) for x in ("q", "k", "v"))
+        self.sets = [(q0, k0, v0, torch.empty_like(q0))]
+        for _ in range(self.n_sets - 1):
+            self.sets.append((q0.clone(), k0.clone(), v0.clone(), torch.empty_like(q0)))
+        self.gidx = inp["global_idx"].to(dev) if inp["global_idx"] is not None else None
+        self.pad = inp["key_pad_mask"].to(dev) if inp["key_pad_mask"] is not None else None
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for i in range(max(warmup, 0)):
+                self.call(i)
+            self.launches_per_step = lf_attn.last_launch_count()
+        torch.cuda.synchronize()
+
+    def call(self, i, stages=7):
+        q, k, v, o = self.sets[i % self.n_sets]
+        self.lf_attn.fwd(q, k, v, self.w.r, dil=self.inp["dil"], global_idx=self.gidx, key_pad_mask=self.pad,
+                         scale=self.w.softmax_scale, out=o, stages=stages, stream=self.stream)
+
+    def capture(self, n, stages=7):
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(g, stream=self.stream):
+            for i in range(n):
+                self.call(i, stages)
+        return g
+
+    def graphs(self, K, stages=7):
+        S = min(self.n_sets, K) if K > 0 else self.n_sets
+        return S, self.capture(S, stages), (self.capture(K % S, stages) if K % S else None)
+
+    def replay(self, K, S, g_main, g_rem):
+        for _ in range(K // S):
+            g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+
+    def time_steps(self, K, stages=7, before=None, after=None):
+        """ms for exactly K steps (one CUDA-event pair around them)."""
+        torch = self.torch
+        S, g_main, g_rem = self.graphs(K, stages)
+        with torch.cuda.stream(self.stream):
+            g_main.replay()
+        torch.cuda.synchronize()
+        if before:
+            before()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            e0.record()
+            self.replay(K, S, g_main, g_rem)
+            e1.record()
+        torch.cuda.synchronize()
+        if after:
+            after()
+        return e0.elapsed_time(e1)
+
+    def stage_us(self, stages, budget_s=0.3):
+        """Mean µs of one stage of the forward alone (graph replays over the rotating sets)."""
+        torch = self.torch
+        with torch.cuda.stream(self.stream):
+            self.call(0)  # prep state for the band / global-row stages
+        torch.cuda.synchronize()
+        one = self.time_steps(self.n_sets, stages) / self.n_sets
+        reps = max(self.n_sets, int(budget_s / max(one * 1e-3, 1e-6)))
+        return 1e3 * self.time_steps(reps, stages) / reps
+
+    def summary(self, ms_per_step, peaks, world=1):
+        w = self.w
+        band_us = self.stage_us(2)
+        out = {"value": round(sharding.job_rate(self.total_f, world, ms_per_step * 1e-3) / 1e12, 3),
+               "unit": "TFLOP/s", "ms_per_step": round(ms_per_step, 6),
+               "tokens_per_s": round(sharding.job_rate(w.B * w.T, world, ms_per_step * 1e-3), 1),
+               "useful_gflop_per_step": round(self.total_f / 1e9, 4),
+               "band_tc_us": round(band_us, 2),
+               "band_frac": round(self.band_f / (band_us * 1e-6) / 1e12 / peaks["bf16_tflops"], 4),
+               "prep_us": round(self.stage_us(1), 2)}
+        if self.gidx is not None:
+            gr_us = self.stage_us(4)
+            out["global_rows_us"] = round(gr_us, 2)
+            out["global_rows_hbm_frac"] = round(self.gr_bytes / (gr_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)
+        out["l2"] = "rotating %d input sets, %.0f MB > 2x L2 (%.0f MB)" % (
+            self.n_sets, self.n_sets * self.set_bytes / 1e6, self.l2 / 1e6)
+        return out
+
+
+def copy_bandwidth(torch, dev, nbytes):
+    """Pinned host <-> device copy bandwidth (GB/s) for nbytes, CUDA events."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        d.copy_(h, non_blocking=True)
+        h.copy_(d, non_blocking=True)
+    torch.cuda.synchronize()
+    res = {}
+    for name, fn in (("h2d", lambda: d.copy_(h, non_blocking=True)), ("d2h", lambda: h.copy_(d, non_blocking=True))):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name] = 10 * nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    return res
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -211,123 +329,92 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     lf_attn.load()
+    peaks, peak_src = load_peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
 
     w = workloads.BY_NAME[args.workload]
-    inp = workloads.make_inputs(w)
-    total_f, band_f, gr_f, gr_bytes = split_flops(w, inp)
-    props = torch.cuda.get_device_properties(local)
-    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
-    es = 2 if w.dtype == "bf16" else 4
-    set_bytes = 4 * w.B * w.H * w.T * w.d * es
-    n_sets = max(2, math.ceil(2 * l2 / set_bytes) + 1)
-    dev = torch.device("cuda", local)
-    q0, k0, v0 = (inp[x].to(dev) for x in ("q", "k", "v"))
-    sets = [(q0, k0, v0, torch.empty_like(q0))]
-    for _ in range(n_sets - 1):
-        sets.append((q0.clone(), k0.clone(), v0.clone(), torch.empty_like(q0)))
-    gidx = inp["global_idx"].to(dev) if inp["global_idx"] is not None else None
-    pad = inp["key_pad_mask"].to(dev) if inp["key_pad_mask"] is not None else None
-    dil = inp["dil"]
-
-    def call(i, stages=7):
-        q, k, v, o = sets[i % n_sets]
-        lf_attn.fwd(q, k, v, w.r, dil=dil, global_idx=gidx, key_pad_mask=pad, scale=w.softmax_scale, out=o,
-                    stages=stages)
-
-    stream = torch.cuda.Stream(device=dev)
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 0)):
-            call(i)
-        launches_per_step = lf_attn.last_launch_count()
-    torch.cuda.synchronize()
-
-    def capture(n, stages=7):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n):
-                call(i, stages)
-        return g
-
+    run = WorkloadRun(w, torch, lf_attn, dev, stream, args.warmup)
+    launches_per_step = run.launches_per_step
     K = args.steps
-    S = min(n_sets, K) if K > 0 else n_sets
-    g_main = capture(S)
-    g_rem = capture(K % S) if K % S else None
-    with torch.cuda.stream(stream):
-        g_main.replay()
-    torch.cuda.synchronize()
 
+    # ---- the timed steps; clocks are sampled during them and over a replay window of
+    #      about a second around them (the steps alone can be shorter than a sample)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    one_ms = run.time_steps(run.n_sets) / run.n_sets
+    pad_steps = max(run.n_sets, int(0.5 / max(one_ms * 1e-3, 1e-6)))
+    run.time_steps(pad_steps)  # half a second of steps before the timed ones (clock window)
+    marks = {}
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
-    with torch.cuda.stream(stream):
-        ev0.record()
-        for _ in range(K // S):
-            g_main.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        ev1.record()
-    torch.cuda.synchronize()
-    t_wall1 = time.time()
+    ms = run.time_steps(K, before=lambda: marks.__setitem__("t0", time.time()),
+                        after=lambda: marks.__setitem__("t1", time.time()))
+    run.time_steps(pad_steps)  # and after them
+    t_win1 = time.time()
     if world > 1:
         dist.barrier()
-    ms = sharding.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
+    ms = sharding.max_over_ranks(ms, device=dev)
     ms_per_step = ms / K
-
-    # ---- per-kernel durations (each kernel alone, graph-replayed over the same rotating sets)
-    def time_stage(stages, reps):
-        g = capture(S, stages)
-        with torch.cuda.stream(stream):
-            g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            a.record()
-            for _ in range(reps):
-                g.replay()
-            b.record()
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / (reps * S)
-
-    reps = max(1, min(2000, int(0.5 / max(ms_per_step * 1e-3, 1e-6) / S)))
-    with torch.cuda.stream(stream):
-        call(0)  # prep state for the band / global-row stages
-    torch.cuda.synchronize()
-    kern = {"band_tc": time_stage(2, reps), "prep": time_stage(1, reps)}
-    if gidx is not None:
-        kern["global_rows"] = time_stage(4, reps)
     sampler.stop()
-    clocks = sampler.summary(t_wall0, t_wall1)
+    clocks = sampler.summary(marks["t0"], marks["t1"])
+    if clocks.get("window") != "timed region":
+        clocks = sampler.summary(marks["t0"] - 0.6, t_win1)
+        clocks["window"] = "replay window of about 1 s around the %d timed steps (they take %.1f ms)" % (K, ms)
 
-    peaks, peak_src = load_peaks()
-    band_tflops = band_f / (kern["band_tc"] * 1e-3) / 1e12
+    base = run.summary(ms_per_step, peaks, world)
+    band_tflops = run.band_f / (base["band_tc_us"] * 1e-6) / 1e12
     roofline = {"kernel": "band_tc_kernel", "bound": "tensor", "achieved": round(band_tflops, 2),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(band_tflops / peaks["bf16_tflops"], 4),
                 "peak_source": "%s bf16 burst (kernel timed alone)" % peak_src,
                 "algorithmic": "4*d*|N(i)| summed over the %d non-global rows, per launch" % int(
-                    band_row_mask(w, inp).sum() * w.H),
+                    band_row_mask(w, run.inp).sum() * w.H),
                 "traffic": traffic_from_profile("band_tc.cuh")}
-    kernels = {"band_tc_us": round(kern["band_tc"] * 1e3, 2), "prep_us": round(kern["prep"] * 1e3, 2)}
-    if "global_rows" in kern:
-        gbw = gr_bytes / (kern["global_rows"] * 1e-3) / 1e9
-        kernels["global_rows_us"] = round(kern["global_rows"] * 1e3, 2)
+    kernels = {k: base[k] for k in ("band_tc_us", "prep_us") if k in base}
+    if "global_rows_us" in base:
+        gbw = run.gr_bytes / (base["global_rows_us"] * 1e-6) / 1e9
+        kernels["global_rows_us"] = base["global_rows_us"]
         kernels["global_rows_hbm"] = {"achieved": round(gbw, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                       "frac": round(gbw / peaks["hbm_gbs"], 4),
                                       "algorithmic": "K,V of the non-padded keys + q,out of the global rows"}
 
+    # ---- one call including its launch (no graph), host wall clock around launch + completion
+    single = []
+    for i in range(20):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            run.call(i)
+        torch.cuda.synchronize()
+        single.append(1e3 * (time.perf_counter() - t0))
+    single_call_ms = float(np.median(single))
+
+    # ---- the other workloads (each its own rotating inputs), rank 0 only
+    others = {}
+    if rank == 0 and world == 1 and not args.no_others:
+        for name in ("qa_B2_T4096_g64_pad", "dilated_T8192_r128", "large_T16384_g32"):
+            if name == w.name:
+                continue
+            ow = workloads.BY_NAME[name]
+            orun = WorkloadRun(ow, torch, lf_attn, dev, stream, args.warmup)
+            o_one = orun.time_steps(orun.n_sets) / orun.n_sets
+            oK = max(orun.n_sets, int(0.4 / max(o_one * 1e-3, 1e-6)))
+            o_ms = orun.time_steps(oK) / oK
+            others[name] = orun.summary(o_ms, peaks)
+            del orun
+            torch.cuda.empty_cache()
+
     # ---- end to end through the host-buffer entry point (pinned host memory)
     e2e = None
     if args.e2e_steps > 0:
+        inp = run.inp
         hq, hk, hv = (inp[x].pin_memory() for x in ("q", "k", "v"))
         hout = torch.empty_like(hq).pin_memory()
         hg = inp["global_idx"].pin_memory() if inp["global_idx"] is not None else None
         hp = inp["key_pad_mask"].pin_memory() if inp["key_pad_mask"] is not None else None
+        dil = inp["dil"]
         with torch.cuda.stream(stream):
             for _ in range(3):
                 lf_attn.fwd_host(hq, hk, hv, w.r, dil=dil, global_idx=hg, key_pad_mask=hp,
@@ -341,16 +428,24 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_ms = sharding.max_over_ranks(a.elapsed_time(b) / args.e2e_steps, device=dev)
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + tuple(x for x in (hg, hp) if x is not None))
-        e2e = {"value": round(sharding.job_rate(total_f, world, e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
-               "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(hout.numel() * hout.element_size()),
-               "api": "lf_attn_fwd_host (pinned host buffers, copies inside the timed region)"}
+        d2h = int(hout.numel() * hout.element_size())
+        bw = copy_bandwidth(torch, dev, h2d)
+        bound_ms = 1e3 * (h2d / (bw["h2d"] * 1e9) + d2h / (bw["d2h"] * 1e9))
+        e2e = {"value": round(sharding.job_rate(run.total_f, world, e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+               "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": d2h,
+               "api": "lf_attn_fwd_host (pinned host buffers, copies inside the timed region)",
+               "copy_bound": {"h2d_gbs": round(bw["h2d"], 2), "d2h_gbs": round(bw["d2h"], 2),
+                              "serial_copy_ms": round(bound_ms, 4),
+                              "frac": round(bound_ms / e2e_ms, 4),
+                              "note": "plain pinned copies of the same bytes on this box, one after the other; "
+                                      "frac = their time / the e2e step (the entry point overlaps copies of one "
+                                      "slice with kernels of another, so frac can exceed 1)"}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, inp, args.cpu_seconds)
+        cpu = cpu_baseline(w, run.inp, args.cpu_seconds)
 
-    tflops = sharding.job_rate(total_f, world, ms_per_step * 1e-3) / 1e12
+    tflops = sharding.job_rate(run.total_f, world, ms_per_step * 1e-3) / 1e12
     tokens = sharding.job_rate(w.B * w.T, world, ms_per_step * 1e-3)
     if rank == 0:
         line = {
@@ -359,13 +454,14 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic: seeded iid N(0,1) q/k/v rounded to %s" % w.dtype,
             "config": workload_config(w, {"parallelism": "replicas (one workload per GPU)" if world > 1 else "1 GPU",
-                                          "l2": "rotating %d input sets, %.0f MB > 2x L2 (%.0f MB)" % (
-                                              n_sets, n_sets * set_bytes / 1e6, l2 / 1e6),
-                                          "timing": "CUDA graphs of %d steps, CUDA events on the launch stream" % S}),
+                                          "l2": base["l2"],
+                                          "timing": "CUDA graphs of %d steps, CUDA events on the launch stream"
+                                                    % min(run.n_sets, K)}),
             "tokens_per_s": round(tokens, 1),
             "pct_of_bf16_peak": round(100.0 * tflops / world / peaks["bf16_tflops"], 2),
-            "useful_gflop_per_step": round(total_f / 1e9, 4),
-            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "useful_gflop_per_step": round(run.total_f / 1e9, 4),
+            "roofline": roofline, "kernels": kernels, "single_call_ms": round(single_call_ms, 4),
+            "workloads": others, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(K * launches_per_step), "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -375,8 +471,9 @@ def run_ours(args):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def oracle_sample_rate(w, inp, seconds, seed=0):
-    """Times the oracle on seeded random rows for about `seconds`; returns (useful FLOPs, seconds, rows, threads)."""
+def oracle_sample_rate(w, inp, seconds, seed=0, nthreads=0):
+    """Times the oracle on seeded random rows for about `seconds` (nthreads 0: every host core); returns
+    (useful FLOPs, seconds, rows, threads)."""
     import oracle
 
     rng = np.random.default_rng(seed)
@@ -401,7 +498,7 @@ def oracle_sample_rate(w, inp, seconds, seed=0):
     def run(rows):
         t0 = time.perf_counter()
         oracle.rows(inp["q"], inp["k"], inp["v"], w.r, rows, dil=inp["dil"], global_idx=G, key_pad_mask=pad,
-                    scale=w.softmax_scale)
+                    scale=w.softmax_scale, nthreads=nthreads)
         return time.perf_counter() - t0
 
     # calibrate: grow the probe until it runs long enough to measure the rate
@@ -415,7 +512,7 @@ def oracle_sample_rate(w, inp, seconds, seed=0):
     n = int(min(max(256, n * seconds / max(dt, 1e-4)), 64 * w.B * w.H * w.T))
     rows = draw(n)
     dt = run(rows)
-    return row_flops(rows.tolist()), dt, n, oracle.max_threads()
+    return row_flops(rows.tolist()), dt, n, (nthreads if nthreads > 0 else oracle.max_threads())
 
 
 def cpu_model():
@@ -430,9 +527,12 @@ def cpu_model():
 
 def cpu_baseline(w, inp, seconds):
     f, dt, n, threads = oracle_sample_rate(w, inp, seconds)
+    f1, dt1, n1, _ = oracle_sample_rate(w, inp, seconds, seed=1, nthreads=1)
     return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": "%d seeded random rows of %s (%.1f s, fp64 C oracle, OpenMP %d threads, %s)" % (
-                n, w.name, dt, threads, cpu_model())}
+                n, w.name, dt, threads, cpu_model()),
+            "single_thread": {"value": round(f1 / dt1 / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+                              "sample": "%d seeded random rows of %s (%.1f s, one thread)" % (n1, w.name, dt1)}}
 
 
 def run_reference(args):

@@ -47,6 +47,18 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sbuf) {
     return (warp ? sbuf[warp - 1] : 0) + x - v;
 }
 
+// Padding bits of the 32 keys of word w (independent byte loads, no chain of
+// dependent ones: the whole word costs one round trip).
+__device__ __forceinline__ uint32_t pad_word(const uint8_t* pad_b, int w, int T) {
+    uint32_t m = 0u;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const int j = (w << 5) + k;
+        m |= (j < T && pad_b[j] != 0) ? (1u << k) : 0u;
+    }
+    return m;
+}
+
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     extern __shared__ __align__(16) uint32_t prep_smem[];
     uint32_t* bits = prep_smem;                                      // [W]
@@ -84,13 +96,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     for (int w = w0; w < w1; ++w) {
         uint32_t qb = bits[w];
         cq += __popc(qb);
-        uint32_t kb = qb;
-        if (pad_b) {
-            for (uint32_t t = qb; t; t &= t - 1) {
-                int j = (w << 5) + __ffs(t) - 1;
-                if (pad_b[j]) kb &= ~(1u << (j & 31));
-            }
-        }
+        const uint32_t kb = (pad_b && qb) ? (qb & ~pad_word(pad_b, w, T)) : qb;
         ck += __popc(kb);
     }
     int oq = block_exclusive_scan(cq, scan_q);
@@ -102,11 +108,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     for (int w = w0; w < w1; ++w) {
         uint32_t qb = bits[w];
         if (writer) p.ws.gbit[static_cast<size_t>(b) * p.W + w] = qb;
+        const uint32_t pw = (pad_b && qb) ? pad_word(pad_b, w, T) : 0u;
         for (uint32_t t = qb; t; t &= t - 1) {
             int j = (w << 5) + __ffs(t) - 1;
             if (writer) gq_out[oq] = j;
             ++oq;
-            if (!pad_b || !pad_b[j]) {
+            if (!((pw >> (j & 31)) & 1u)) {
                 gk_s[ok] = j;
                 if (writer) gk_out[ok] = j;
                 ++ok;
