@@ -191,8 +191,10 @@ int lf_attn_band_plan(int B, int H, int T, int r, const int32_t* dil, int n_glob
  *   the caller still provides q, k, v, out, global_idx and key_pad_mask.
  *   Returns LF_ERR_SCRATCH_TOO_SMALL, before launching anything, when these
  *   sizes need more than 32 MiB - 256 bytes of workspace (the
- *   lf_attn_workspace_bytes figure); the five reference workloads need at
- *   most about 9 MiB.
+ *   lf_attn_workspace_bytes figure).  bf16 sizes need about 19 MiB for
+ *   the band kernel's fixed partial-state slots (two per CTA, 296 CTAs)
+ *   plus what grows with B, H, T and n_global: 19 to 26 MiB for the sizes
+ *   the tests use (up to B = 2, H = 16, T = 16384, 64 global tokens).
  *   The first call on a device sets that device up (kernel attributes and
  *   the scratch array's device address); make that first call before any
  *   stream capture.

@@ -139,10 +139,11 @@ def test_many_global_rows_span_several_row_groups():
 
 
 def test_score_jumps_inside_a_key_block():
-    """Every 128 keys, the last quarter has 16x the norm, so inside one key
-    block a row's scaled score jumps by far more than 2^64 after its first
-    columns were already exponentiated: the band kernel must rescale the
-    probabilities it already holds, and O, in place."""
+    """Every 128 keys, the last quarter has 16x the norm, so within one
+    64-key block a row's scaled scores jump by far more than 2^8 over the
+    exponent base the earlier blocks set: the band kernel must move the base
+    to the block's max before exponentiating it and rescale O and the row
+    sum in place."""
     w = workloads.custom("spikes", "bf16", 1, 2, 700, 64, 200, dil=[1, 3], globals_per_b=[[5]], scale=1.0,
                          seed=39)
     inp = workloads.make_inputs(w)
