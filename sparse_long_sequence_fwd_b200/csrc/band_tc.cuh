@@ -519,17 +519,45 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
     }
 }
 
-// Writes y = O * inv as bf16 to dst (16-byte stores).
-__device__ __forceinline__ void store_row(__nv_bfloat16* dst, const float* o, float inv) {
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
+// Writes output dimensions [32 hd, 32 hd + 32) of the warp's 32 rows as
+// bf16: y = o * inv for this lane's row (32 values) to row_ptr + 32 hd when
+// `write`.  Every store instruction writes whole 64-byte row halves, eight of
+// them: each group of 4 lanes transposes its 4 x 4 block of 16-byte chunks
+// with two rounds of xor shuffles, after which store e of lane 4g + j writes
+// chunk j of row 4g + e.  (One lane per row would make every store touch 32
+// lines.)  Warp-wide: every lane calls it.
+__device__ __forceinline__ void store_half_rows(__nv_bfloat16* row_ptr, bool write, int hd, const float* o,
+                                                float inv) {
+    const int lane = threadIdx.x & 31;
+    uint32_t x[4][4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        uint4 v;
-        v.x = pack_bf16x2(o[8 * u + 0] * inv, o[8 * u + 1] * inv);
-        v.y = pack_bf16x2(o[8 * u + 2] * inv, o[8 * u + 3] * inv);
-        v.z = pack_bf16x2(o[8 * u + 4] * inv, o[8 * u + 5] * inv);
-        v.w = pack_bf16x2(o[8 * u + 6] * inv, o[8 * u + 7] * inv);
-        d4[u] = v;
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) x[c][w] = pack_bf16x2(o[8 * c + 2 * w] * inv, o[8 * c + 2 * w + 1] * inv);
+#pragma unroll
+    for (int sh = 2; sh >= 1; sh >>= 1) {
+        const bool upper = (lane & sh) != 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (e & sh) continue;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t send = upper ? x[e][w] : x[e + sh][w];
+                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, sh);
+                if (upper)
+                    x[e][w] = recv;
+                else
+                    x[e + sh][w] = recv;
+            }
+        }
+    }
+    const int g0 = lane & ~3, j = lane & 3;
+    const unsigned long long rp = reinterpret_cast<unsigned long long>(row_ptr + 32 * hd);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const unsigned long long dst = __shfl_sync(0xffffffffu, rp, g0 + e);
+        const int wr = __shfl_sync(0xffffffffu, write ? 1 : 0, g0 + e);
+        if (wr) *reinterpret_cast<uint4*>(dst + 16ull * j) = make_uint4(x[e][0], x[e][1], x[e][2], x[e][3]);
     }
 }
 
@@ -542,7 +570,8 @@ __device__ __forceinline__ float* part_slot(const BandTcParams& p, int s, int ts
 
 // Output of a finished piece (warp-wide: every lane calls it): its
 // descriptor d stays in shared memory until this is done; m and l are this
-// thread's row's exponent base and sum.
+// thread's row's exponent base and sum.  The row is handled 32 output
+// dimensions at a time (registers: this runs with the next piece's state live).
 __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiece* d, float m, float l, uint32_t tO,
                                           int wq, int ticket, volatile int* abort_flag) {
     const int lane = threadIdx.x & 31;
@@ -553,17 +582,22 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
     bool write = ip < Tc;
     if (write) write = !((p.gbit[static_cast<size_t>(d->b) * p.W + (i >> 5)] >> (i & 31)) & 1u);
     __nv_bfloat16* dst = p.out + (static_cast<size_t>(d->bh) * p.T + (write ? i : 0)) * kHD;
-    float o[64];
-    {
-        uint32_t r[64];
-        tmem_ld64(tO, r);
+    // 32 columns of this row's O (dimensions [32 hd, 32 hd + 32))
+    auto load_o = [&](int hd, float* o) {
+        uint32_t r[32];
+        tmem_ld32(tO + 32u * hd, r);
         tmem_ld_wait(r);
-        reg_fence32(r + 32);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) o[c] = __uint_as_float(r[c]);
-    }
+        for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(r[c]);
+    };
     if (d->blk_lo == 0 && d->blk_hi == d->nbb + d->ngb) {  // the whole tile
-        if (write) store_row(dst, o, l > 0.f ? 1.f / l : 0.f);
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int hd = 0; hd < 2; ++hd) {
+            float o[32];
+            load_o(hd, o);
+            store_half_rows(dst, write, hd, o, inv);
+        }
         return;
     }
     const int s0 = d->s0, s1 = d->s1;
@@ -573,8 +607,14 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
     if (ticket < npieces - 1) {  // not the last to arrive: leave the partial state for the last
         float* slot = part_slot(p, self, tstart);
         float4* o4 = reinterpret_cast<float4*>(slot);
+#pragma unroll 1
+        for (int hd = 0; hd < 2; ++hd) {
+            float o[32];
+            load_o(hd, o);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) o4[u * kBM + x] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+            for (int u = 0; u < 8; ++u)
+                o4[(8 * hd + u) * kBM + x] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        }
         slot[kBM * kHD + x] = m;
         slot[kBM * kHD + kBM + x] = l;
         red_release_add(cnt + 1, 1);  // each lane: its stores, then its count (no wait)
@@ -597,15 +637,10 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
     }
     // M = max of the pieces' bases; y = sum_s w_s O_s / sum_s w_s l_s with w_s = 2^(m_s - M),
     // summed in CTA order whichever piece merges (the same operations either way)
-    float acc[64];
-    float L = 0.f;
-    if (npieces == 2 && ok) {  // the common case: one other piece, all its loads at once
+    if (npieces == 2 && ok) {  // the common case: one other piece
         const int so = self == s0 ? s1 : s0;
         const float* slot = part_slot(p, so, tstart);
         const float4* o4 = reinterpret_cast<const float4*>(slot);
-        float4 v[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] = __ldcg(o4 + u * kBM + x);
         const float mo = __ldcg(slot + kBM * kHD + x);
         const float lo = __ldcg(slot + kBM * kHD + kBM + x);
         const float M = fmaxf(m, mo);
@@ -614,48 +649,73 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
         const float wo = mo == -INFINITY ? 0.f : ex2_approx(mo - Mu);
         const bool self_first = self == s0;
         const float w1 = self_first ? ws : wo, w2 = self_first ? wo : ws;
-        L = fmaf(w2, self_first ? lo : l, w1 * (self_first ? l : lo));
+        const float L = fmaf(w2, self_first ? lo : l, w1 * (self_first ? l : lo));
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll 1
+        for (int hd = 0; hd < 2; ++hd) {
+            float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const float a0 = v[u].x, a1 = v[u].y, a2 = v[u].z, a3 = v[u].w;
-            const float b0 = o[4 * u], b1 = o[4 * u + 1], b2 = o[4 * u + 2], b3 = o[4 * u + 3];
-            acc[4 * u] = fmaf(w2, self_first ? a0 : b0, w1 * (self_first ? b0 : a0));
-            acc[4 * u + 1] = fmaf(w2, self_first ? a1 : b1, w1 * (self_first ? b1 : a1));
-            acc[4 * u + 2] = fmaf(w2, self_first ? a2 : b2, w1 * (self_first ? b2 : a2));
-            acc[4 * u + 3] = fmaf(w2, self_first ? a3 : b3, w1 * (self_first ? b3 : a3));
+            for (int u = 0; u < 8; ++u) v[u] = __ldcg(o4 + (8 * hd + u) * kBM + x);
+            float o[32];
+            load_o(hd, o);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float a[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float b = o[4 * u + k];
+                    o[4 * u + k] = fmaf(w2, self_first ? a[k] : b, w1 * (self_first ? b : a[k]));
+                }
+            }
+            store_half_rows(dst, write, hd, o, inv);
         }
     } else {
         float M = m;
         for (int s = s0; s <= s1; ++s)
             if (s != self && ok) M = fmaxf(M, __ldcg(part_slot(p, s, tstart) + kBM * kHD + x));
         const float Mu = M == -INFINITY ? 0.f : M;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+        float L = 0.f;
         for (int s = s0; s <= s1; ++s) {
             if (s == self) {
-                const float wv = m == -INFINITY ? 0.f : ex2_approx(m - Mu);
-                L = fmaf(wv, l, L);
-#pragma unroll
-                for (int c = 0; c < 64; ++c) acc[c] = fmaf(wv, o[c], acc[c]);
-                continue;
-            }
-            if (!ok) continue;
-            const float* slot = part_slot(p, s, tstart);
-            const float ms = __ldcg(slot + kBM * kHD + x);
-            const float wv = ms == -INFINITY ? 0.f : ex2_approx(ms - Mu);
-            L = fmaf(wv, __ldcg(slot + kBM * kHD + kBM + x), L);
-            const float4* o4 = reinterpret_cast<const float4*>(slot);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const float4 v = __ldcg(o4 + u * kBM + x);
-                acc[4 * u] = fmaf(wv, v.x, acc[4 * u]);
-                acc[4 * u + 1] = fmaf(wv, v.y, acc[4 * u + 1]);
-                acc[4 * u + 2] = fmaf(wv, v.z, acc[4 * u + 2]);
-                acc[4 * u + 3] = fmaf(wv, v.w, acc[4 * u + 3]);
+                L = fmaf(m == -INFINITY ? 0.f : ex2_approx(m - Mu), l, L);
+            } else if (ok) {
+                const float* slot = part_slot(p, s, tstart);
+                const float ms = __ldcg(slot + kBM * kHD + x);
+                L = fmaf(ms == -INFINITY ? 0.f : ex2_approx(ms - Mu), __ldcg(slot + kBM * kHD + kBM + x), L);
             }
         }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll 1
+        for (int hd = 0; hd < 2; ++hd) {
+            float acc[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+            for (int s = s0; s <= s1; ++s) {
+                if (s == self) {
+                    const float wv = m == -INFINITY ? 0.f : ex2_approx(m - Mu);
+                    float o[32];
+                    load_o(hd, o);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) acc[c] = fmaf(wv, o[c], acc[c]);
+                    continue;
+                }
+                if (!ok) continue;
+                const float* slot = part_slot(p, s, tstart);
+                const float ms = __ldcg(slot + kBM * kHD + x);
+                const float wv = ms == -INFINITY ? 0.f : ex2_approx(ms - Mu);
+                const float4* o4 = reinterpret_cast<const float4*>(slot);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float4 v = __ldcg(o4 + (8 * hd + u) * kBM + x);
+                    acc[4 * u] = fmaf(wv, v.x, acc[4 * u]);
+                    acc[4 * u + 1] = fmaf(wv, v.y, acc[4 * u + 1]);
+                    acc[4 * u + 2] = fmaf(wv, v.z, acc[4 * u + 2]);
+                    acc[4 * u + 3] = fmaf(wv, v.w, acc[4 * u + 3]);
+                }
+            }
+            store_half_rows(dst, write, hd, acc, inv);
+        }
     }
-    if (write) store_row(dst, acc, L > 0.f ? 1.f / L : 0.f);
     __syncwarp();
     if (lane == 0) {  // ready for the next call
         cnt[0] = 0;
@@ -709,30 +769,27 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     // written; its descriptor slot is released (Q-empty) only then.
     int prev_slot = -1;
     float m_prev = 0.f, l_prev = 0.f;
-    int ticket = 0;  // merge ticket of the previous piece (split pieces)
+    int ticket = 0;       // merge ticket of the current piece (split pieces), taken at its last block
+    int ticket_prev = 0;  // the previous piece's, kept until its rows are written
     auto finish_prev = [&]() {
         const BandPiece* dq = reinterpret_cast<const BandPiece*>(smem + kOffDesc + prev_slot * kDescBytes);
-        flush_rows(p, dq, m_prev, l_prev, tO, wq, __shfl_sync(0xffffffffu, ticket, 0), abort_flag);
+        flush_rows(p, dq, m_prev, l_prev, tO, wq, __shfl_sync(0xffffffffu, ticket_prev, 0), abort_flag);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarQEmpty + prev_slot]);
         prev_slot = -1;
     };
     for (;;) {
-        // the previous piece's O is final once its last product is done: its rows
-        // (one place in the code for every piece, the last one included)
-        if (prev_slot >= 0) {
-            if (!wait_product(g - 1)) return;
-            need_prep();
-            finish_prev();
-        }
-        if (done) break;
-        // the piece's descriptor, published by the producer with its Q tile
+        // After the last piece, one more pass with no piece (one empty block)
+        // writes that piece's rows.
+        const bool have = !done;
         const uint32_t qs = qt & 1u;
-        if (!wait_warp(&bars[kBarQFull + qs], (qt >> 1) & 1u)) return;
-        ++qt;
+        if (have) {  // the piece's descriptor, published by the producer with its Q tile
+            if (!wait_warp(&bars[kBarQFull + qs], (qt >> 1) & 1u)) return;
+            ++qt;
+        }
         const BandPiece* dp = reinterpret_cast<const BandPiece*>(smem + kOffDesc + qs * kDescBytes);
-        done = dp->last != 0;
-        const int blk_lo = dp->blk_lo, blk_hi = dp->blk_hi, nbb = dp->nbb;
+        if (have) done = dp->last != 0;
+        const int blk_lo = have ? dp->blk_lo : 0, blk_hi = have ? dp->blk_hi : 1, nbb = dp->nbb;
         const int i = dp->c + dp->dil * (dp->q0 + x);  // this row's position in the sequence
         // Band blocks inside every row's window and inside [0, Tc) need no mask:
         // 0 <= 64 kb + y - x <= 2r for all x < 128, y < 64, and 0 <= j0, j0 + 64 <= Tc.
@@ -750,140 +807,152 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
         float m_ref = -INFINITY;  // exponent base (scaled, log2 domain; -inf: nothing kept yet)
         float l_row = 0.f;        // row sum relative to m_ref
 #pragma unroll 1
-        for (int blk = blk_lo; blk < blk_hi; ++blk, ++g) {
+        for (int blk = blk_lo; blk < blk_hi; ++blk) {
             const uint32_t b = g % kSBufs;
-            // ---- which columns this row keeps (bit j of mk[c]: column 32 c + j)
-            uint32_t mk[2] = {0xffffffffu, 0xffffffffu};
-            bool live0 = true, live1 = true, full0 = true, full1 = true;
-            if (blk < ib_lo || blk >= ib_hi) {
-                if (blk < nbb) {
-                    const int kb = dp->kb_lo + blk;
-                    const int Tc = dp->Tc;
-                    const int j0 = dp->kbase + kBN * kb;
-                    // kept columns [ylo, yhi): the window and [0, Tc)
-                    const int ylo = max(max(0, x - kBN * kb), -j0);
-                    const int yhi = min(min(kBN, x + 2 * p.r + 1 - kBN * kb), Tc - j0);
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t m = range_bits(ylo - 32 * c, yhi - 32 * c);
-                        if (p.pad) {
-                            const int jd = j0 + 32 * c + lane;
-                            const bool padded =
-                                jd >= 0 && jd < Tc &&
-                                p.pad[static_cast<size_t>(dp->b) * p.T + dp->c + static_cast<size_t>(dp->dil) * jd] != 0;
-                            m &= ~__ballot_sync(0xffffffffu, padded);
-                        }
-                        mk[c] = m;
-                    }
-                } else {  // global keys not already in the row's window
-                    const int bs = dp->b;
-                    if (bs != gk_b) {
-                        need_prep();
-                        gk_b = bs;
-                        ngk = *reinterpret_cast<const volatile int*>(p.n_gk + bs);
-                        const int32_t* gl = p.gk_list + static_cast<size_t>(bs) * p.gstride;
-                        gk_reg[0] = lane < ngk ? static_cast<uint32_t>(gl[lane]) : 0u;
-                        gk_reg[1] = 32 + lane < ngk ? static_cast<uint32_t>(gl[32 + lane]) : 0u;
-                    }
-                    const int gb = blk - nbb;
-                    const int nvalid = min(kBN, ngk - gb * kBN);
-                    const int32_t* gkl = p.gk_list + static_cast<size_t>(bs) * p.gstride + gb * kBN;
-                    const int dil = dp->dil, reach = dil * p.r;
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t m = 0u;
-                        const int na = min(32, nvalid - 32 * c);
-                        if (na > 0) {
-                            const uint32_t kc = gb == 0 ? gk_reg[c] : (lane < na ? static_cast<uint32_t>(gkl[32 * c + lane]) : 0u);
-#pragma unroll 1
-                            for (int a = 0; a < na; ++a) {
-                                const int diff = static_cast<int>(__shfl_sync(0xffffffffu, kc, a)) - i;
-                                const bool in_window = diff <= reach && diff >= -reach && (dil == 1 || diff % dil == 0);
-                                m |= in_window ? 0u : (1u << a);
-                            }
-                        }
-                        mk[c] = m;
-                    }
-                }
-                live0 = __any_sync(0xffffffffu, mk[0] != 0u);
-                live1 = __any_sync(0xffffffffu, mk[1] != 0u);
-                full0 = __all_sync(0xffffffffu, mk[0] == 0xffffffffu);
-                full1 = __all_sync(0xffffffffu, mk[1] == 0xffffffffu);
-            }
-
-            if (split && blk == blk_hi - 1) {  // the merge ticket, while this last block is computed
-                need_prep();                     // (prep zeroes the tickets)
-                if (lane == 0) ticket = atomicAdd(p.cnt + (static_cast<size_t>(dp->tile) * 4 + wq) * 2, 1);
-            }
-
-            // ---- the row's 64 scores
-            if (!wait_warp(&bars[kBarSFull + b], (g / kSBufs) & 1u)) return;
-            tc_fence_after();
             const uint32_t tS = tmem_base + lane_off + 64u * b;
-            uint32_t s[64];
-            tmem_ld64(tS, s);
-            tmem_ld_wait(s);
-            reg_fence32(s + 32);
-
-            // ---- mask and block max (scaled: the largest kept s * kmul)
-            float mx0 = -INFINITY, mx1 = -INFINITY;
-            if (live0) {
-                if (!full0) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (!((mk[0] >> j) & 1u)) s[j] = fill;
-                }
-                mx0 = (pos ? max32(s) : min32(s)) * kmul;
-            }
-            if (live1) {
-                if (!full1) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (!((mk[1] >> j) & 1u)) s[32 + j] = fill;
-                }
-                mx1 = (pos ? max32(s + 32) : min32(s + 32)) * kmul;
-            }
-            const float mxs = fmaxf(mx0, mx1);
-            // ---- exponent base
             float alpha = 1.f;
             bool o_move = false;
-            if (m_ref == -INFINITY) {
-                m_ref = mxs;  // nothing held so far (the row's O and l are 0)
-            } else if (mxs > m_ref + kRescaleLog2) {
-                alpha = ex2_approx(m_ref - mxs);
-                l_row *= alpha;
-                m_ref = mxs;
-                o_move = true;
-            }
-            const float nb2 = m_ref == -INFINITY ? 0.f : -m_ref;
-
-            // ---- p = 2^(s * kmul - base), row sums, bf16 pairs
-            uint32_t pk[32];
-            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
-            const float2 k2 = make_float2(kmul, kmul), b2 = make_float2(nb2, nb2);
+            if (have) {
+                // ---- which columns this row keeps (bit j of mk[c]: column 32 c + j)
+                uint32_t mk[2] = {0xffffffffu, 0xffffffffu};
+                bool live0 = true, live1 = true, full0 = true, full1 = true;
+                if (blk < ib_lo || blk >= ib_hi) {
+                    if (blk < nbb) {
+                        const int kb = dp->kb_lo + blk;
+                        const int Tc = dp->Tc;
+                        const int j0 = dp->kbase + kBN * kb;
+                        // kept columns [ylo, yhi): the window and [0, Tc)
+                        const int ylo = max(max(0, x - kBN * kb), -j0);
+                        const int yhi = min(min(kBN, x + 2 * p.r + 1 - kBN * kb), Tc - j0);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                if (c == 0 ? live0 : live1) {
+                        for (int c = 0; c < 2; ++c) {
+                            uint32_t m = range_bits(ylo - 32 * c, yhi - 32 * c);
+                            if (p.pad) {
+                                const int jd = j0 + 32 * c + lane;
+                                const bool padded =
+                                    jd >= 0 && jd < Tc &&
+                                    p.pad[static_cast<size_t>(dp->b) * p.T + dp->c + static_cast<size_t>(dp->dil) * jd] != 0;
+                                m &= ~__ballot_sync(0xffffffffu, padded);
+                            }
+                            mk[c] = m;
+                        }
+                    } else {  // global keys not already in the row's window
+                        const int bs = dp->b;
+                        if (bs != gk_b) {
+                            need_prep();
+                            gk_b = bs;
+                            ngk = *reinterpret_cast<const volatile int*>(p.n_gk + bs);
+                            const int32_t* gl = p.gk_list + static_cast<size_t>(bs) * p.gstride;
+                            gk_reg[0] = lane < ngk ? static_cast<uint32_t>(gl[lane]) : 0u;
+                            gk_reg[1] = 32 + lane < ngk ? static_cast<uint32_t>(gl[32 + lane]) : 0u;
+                        }
+                        const int gb = blk - nbb;
+                        const int nvalid = min(kBN, ngk - gb * kBN);
+                        const int32_t* gkl = p.gk_list + static_cast<size_t>(bs) * p.gstride + gb * kBN;
+                        const int dil = dp->dil, reach = dil * p.r;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const float2 t0 = ffma2(make_float2(__uint_as_float(s[32 * c + j]), __uint_as_float(s[32 * c + j + 1])), k2, b2);
-                        const float2 t1 = ffma2(make_float2(__uint_as_float(s[32 * c + j + 2]), __uint_as_float(s[32 * c + j + 3])), k2, b2);
-                        const float2 e0 = make_float2(ex2_approx(t0.x), ex2_approx(t0.y));
-                        const float2 e1 = make_float2(ex2_approx(t1.x), ex2_approx(t1.y));
-                        acc0 = fadd2(acc0, e0);
-                        acc1 = fadd2(acc1, e1);
-                        pk[16 * c + j / 2] = pack_bf16x2(e0.x, e0.y);
-                        pk[16 * c + j / 2 + 1] = pack_bf16x2(e1.x, e1.y);
+                        for (int c = 0; c < 2; ++c) {
+                            uint32_t m = 0u;
+                            const int na = min(32, nvalid - 32 * c);
+                            if (na > 0) {
+                                const uint32_t kc = gb == 0 ? gk_reg[c] : (lane < na ? static_cast<uint32_t>(gkl[32 * c + lane]) : 0u);
+#pragma unroll 1
+                                for (int a = 0; a < na; ++a) {
+                                    const int diff = static_cast<int>(__shfl_sync(0xffffffffu, kc, a)) - i;
+                                    const bool in_window = diff <= reach && diff >= -reach && (dil == 1 || diff % dil == 0);
+                                    m |= in_window ? 0u : (1u << a);
+                                }
+                            }
+                            mk[c] = m;
+                        }
                     }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) pk[16 * c + j] = 0u;
+                    live0 = __any_sync(0xffffffffu, mk[0] != 0u);
+                    live1 = __any_sync(0xffffffffu, mk[1] != 0u);
+                    full0 = __all_sync(0xffffffffu, mk[0] == 0xffffffffu);
+                    full1 = __all_sync(0xffffffffu, mk[1] == 0xffffffffu);
                 }
-            }
-            l_row += (acc0.x + acc0.y) + (acc1.x + acc1.y);
 
-            // ---- P over S; O is rescaled only once the previous product is done
-            tmem_st32(tS, pk);
+                if (split && blk == blk_hi - 1) {  // the merge ticket, while this last block is computed
+                    need_prep();                     // (prep zeroes the tickets)
+                    if (lane == 0) ticket = atomicAdd(p.cnt + (static_cast<size_t>(dp->tile) * 4 + wq) * 2, 1);
+                }
+
+                // ---- the row's 64 scores
+                if (!wait_warp(&bars[kBarSFull + b], (g / kSBufs) & 1u)) return;
+                tc_fence_after();
+                uint32_t s[64];
+                tmem_ld64(tS, s);
+                tmem_ld_wait(s);
+                reg_fence32(s + 32);
+
+                // ---- mask and block max (scaled: the largest kept s * kmul)
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+                if (live0) {
+                    if (!full0) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (!((mk[0] >> j) & 1u)) s[j] = fill;
+                    }
+                    mx0 = (pos ? max32(s) : min32(s)) * kmul;
+                }
+                if (live1) {
+                    if (!full1) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (!((mk[1] >> j) & 1u)) s[32 + j] = fill;
+                    }
+                    mx1 = (pos ? max32(s + 32) : min32(s + 32)) * kmul;
+                }
+                const float mxs = fmaxf(mx0, mx1);
+                // ---- exponent base
+                if (m_ref == -INFINITY) {
+                    m_ref = mxs;  // nothing held so far (the row's O and l are 0)
+                } else if (mxs > m_ref + kRescaleLog2) {
+                    alpha = ex2_approx(m_ref - mxs);
+                    l_row *= alpha;
+                    m_ref = mxs;
+                    o_move = true;
+                }
+                const float nb2 = m_ref == -INFINITY ? 0.f : -m_ref;
+
+                // ---- p = 2^(s * kmul - base), row sums, bf16 pairs
+                uint32_t pk[32];
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+                const float2 k2 = make_float2(kmul, kmul), b2 = make_float2(nb2, nb2);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    if (c == 0 ? live0 : live1) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float2 t0 = ffma2(make_float2(__uint_as_float(s[32 * c + j]), __uint_as_float(s[32 * c + j + 1])), k2, b2);
+                            const float2 t1 = ffma2(make_float2(__uint_as_float(s[32 * c + j + 2]), __uint_as_float(s[32 * c + j + 3])), k2, b2);
+                            const float2 e0 = make_float2(ex2_approx(t0.x), ex2_approx(t0.y));
+                            const float2 e1 = make_float2(ex2_approx(t1.x), ex2_approx(t1.y));
+                            acc0 = fadd2(acc0, e0);
+                            acc1 = fadd2(acc1, e1);
+                            pk[16 * c + j / 2] = pack_bf16x2(e0.x, e0.y);
+                            pk[16 * c + j / 2 + 1] = pack_bf16x2(e1.x, e1.y);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) pk[16 * c + j] = 0u;
+                    }
+                }
+                l_row += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+
+                // ---- P over S (released to the MMA below)
+                tmem_st32(tS, pk);
+            }
+            // ---- the previous piece's rows, once its last product is done.  This
+            // block's P is held back until they are written (the first product
+            // of a piece overwrites O), so the wait overlaps this block's work.
+            if (prev_slot >= 0) {
+                if (!wait_product(g - 1)) return;
+                need_prep();
+                finish_prev();
+            }
+            if (!have) break;
+            // ---- O is rescaled only once the previous product is done
             if (__any_sync(0xffffffffu, o_move)) {
                 if (!wait_product(g - 1)) return;
                 rescale_o(tO, alpha);
@@ -892,11 +961,14 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[kBarPFull + b]);
+            ++g;
         }
-        // ---- this piece's rows are written once its last product is done
+        if (!have) break;
+        // ---- this piece's rows are written during the next piece's first block
         prev_slot = static_cast<int>(qs);
         m_prev = m_ref;
         l_prev = l_row;
+        ticket_prev = ticket;
     }
 }
 

@@ -153,6 +153,39 @@ def test_score_jumps_inside_a_key_block():
     parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
 
 
+def _split_then_one_block_split(B, H, T, r, dil, n_global):
+    """Pairs of pieces the band kernel processes back to back in one CTA: a
+    split piece, then a split piece of one block (its merge ticket is taken in
+    the same block that writes the first piece's rows).  Each CTA processes the
+    split tile at the end of its range first, then the range from its start."""
+    plan = lf_attn.band_plan(B, H, T, r, dil=dil, n_global=n_global).tolist()
+    by_cta = {}
+    for pc in plan:
+        by_cta.setdefault(pc[0], []).append(pc)
+    split = lambda pc: pc[2] > 0 or pc[3] < pc[4]
+    hits = 0
+    for pieces in by_cta.values():
+        order = pieces
+        if len(pieces) >= 2 and pieces[-1][3] < pieces[-1][4]:
+            order = [pieces[-1]] + pieces[:-1]
+        hits += sum(1 for a, b in zip(order, order[1:]) if split(a) and split(b) and b[3] - b[2] == 1)
+    return hits
+
+
+@pytest.mark.parametrize("dil,n_random", [([1] * 6 + [2] * 6, 3), ([1, 2, 3, 4] * 2, 5)])
+def test_split_piece_then_one_block_split_piece(dil, n_random):
+    """A CTA writes a split piece's rows while it computes the next piece's
+    first block; when that next piece is a split piece of one block, both
+    pieces' merge tickets are live at once.  The sizes are chosen so the work
+    split has many such pairs (checked on the host), and every element is
+    compared with the oracle."""
+    H, T, r = len(dil), 2000 if len(dil) == 12 else 1500, 64
+    w = workloads.custom("split_pairs_h%d" % H, "bf16", 1, H, T, 64, r, dil=dil, n_random_globals=n_random, seed=44)
+    inp = workloads.make_inputs(w)
+    assert _split_then_one_block_split(1, H, T, r, dil, int(inp["global_idx"].shape[-1])) > 0
+    parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
+
+
 def test_out_of_range_global_entries_are_ignored_and_flagged():
     w = workloads.custom("bad_g", "bf16", 1, 2, 300, 64, 20, seed=40)
     inp = workloads.make_inputs(w)
