@@ -193,8 +193,8 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
 // and cpc consecutive 128-key chunks of the key axis.  The chunks of K and V
 // stream through a two-stage ring in padded shared memory (cp.async,
 // zero-filled past T); the first two are requested before anything that
-// depends on the prep kernel (the global-query count and list, the query
-// rows), so the HBM latency overlaps those reads.  Every warp forms
+// depends on the prep kernel (the global-query count and the query rows,
+// which prep packs in list order), so the HBM latency overlaps those reads.  Every warp forms
 // S = Q K^T (16 x 128, fp32 in registers), applies the key padding mask,
 // runs the online softmax (log2 domain, exp2) and accumulates O += P V with
 // P re-packed from the S registers as bf16 A fragments and V fragments from
@@ -245,7 +245,6 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
     const size_t base = static_cast<size_t>(bh) * T * 64;
     const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(p.k) + base;
     const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(p.v) + base;
-    const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(p.q) + base;
     const int nblk = (T + kGrKeys - 1) / kGrKeys;
     const int c_lo = split * p.cpc, c_hi = min(nblk, c_lo + p.cpc);
 
@@ -267,21 +266,16 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
     if (c_lo + 1 < c_hi) issue(c_lo + 1, 1);
     cp_async_commit();
 
-    const int nq = p.ws.n_gq[b];
+    // Q fragments of rows row0 + g8 and row0 + g8 + 8 from the packed global
+    // queries (prep's output: zero past the sample's count, so no count or list
+    // is needed first), loaded alongside the count
     const int row0 = blockIdx.z * kGrRows + warp * 16;  // this warp's first global-row slot
-    if (blockIdx.z * kGrRows >= nq) {
-        cp_async_wait<0>();  // no copy may still target this CTA's shared memory
-        return;
-    }
-    const int32_t* gq = p.ws.gq_list + static_cast<size_t>(b) * p.gstride;
-    const bool active = row0 < nq;
-
-    // Q fragments of rows row0 + g8 and row0 + g8 + 8 (zero past nq)
     uint32_t qa[4][4];
     {
+        const __nv_bfloat16* qgb = p.ws.qg + static_cast<size_t>(bh) * p.ngp * 64;
         const int ra = row0 + g8, rb = row0 + g8 + 8;
-        const __nv_bfloat16* qra = ra < nq ? qb + static_cast<size_t>(gq[ra]) * 64 : nullptr;
-        const __nv_bfloat16* qrb = rb < nq ? qb + static_cast<size_t>(gq[rb]) * 64 : nullptr;
+        const __nv_bfloat16* qra = ra < p.ngp ? qgb + static_cast<size_t>(ra) * 64 : nullptr;
+        const __nv_bfloat16* qrb = rb < p.ngp ? qgb + static_cast<size_t>(rb) * 64 : nullptr;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
             const int c0 = 16 * ks + 2 * t4;
@@ -291,6 +285,12 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
             qa[ks][3] = qrb ? *reinterpret_cast<const uint32_t*>(qrb + c0 + 8) : 0u;
         }
     }
+    const int nq = p.ws.n_gq[b];
+    if (blockIdx.z * kGrRows >= nq) {
+        cp_async_wait<0>();  // no copy may still target this CTA's shared memory
+        return;
+    }
+    const bool active = row0 < nq;
     float o[8][4];
 #pragma unroll
     for (int nd = 0; nd < 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
@@ -298,6 +298,10 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
     const float sl2 = p.sl2;
 
     for (int ch = c_lo; ch < c_hi; ++ch) {
+        // the merge kernel may launch once every CTA is on its last chunk (it
+        // waits for this whole grid before reading): its launch overlaps that
+        // chunk without its CTAs sitting resident through the earlier ones
+        if (ch == c_hi - 1) grid_dep_launch();
         const int st = (ch - c_lo) & 1;
         const __nv_bfloat16* Ks = gr_ring + st * 2 * kGrChunkElems;
         const __nv_bfloat16* Vs = Ks + kGrChunkElems;
@@ -419,9 +423,9 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
 // One CTA per (global-row slot, b*h), one thread per output column: the
 // splits' partial states combine as M = max_c m_c, w_c = 2^(m_c - M),
 // y = sum_c w_c acc_c / sum_c w_c l_c.  Launched as the split kernel's
-// programmatic dependent (its launch overlaps the splits' end).  Every load
-// of a pass is issued before any of its values is used, so each pass costs
-// one round trip to L2.
+// programmatic dependent: the split kernel lets it launch once every split
+// CTA is on its last chunk, so only griddepcontrol.wait separates the two.  All
+// its loads are issued before any value is used (one round trip to L2).
 __global__ void __launch_bounds__(64) global_rows_merge_kernel(const __grid_constant__ GlobalRowParams p) {
     __shared__ float wsh[kMaxSplits];
     __shared__ float red[2];
@@ -433,9 +437,14 @@ __global__ void __launch_bounds__(64) global_rows_merge_kernel(const __grid_cons
     const float* src = p.ws.partial + (static_cast<size_t>(bh) * p.gstride + a) * nsplit * 66;
     const int32_t g = p.ws.gq_list[static_cast<size_t>(b) * p.gstride + a];
 
-    // pass 1: every split's (m, l); thread c holds split c (nsplit <= 64)
+    // every load first, so the whole merge costs one round trip to L2: split
+    // c's (m, l) in thread c (nsplit <= 64), and column tid of every split
     const float mc = tid < nsplit ? __ldcg(src + static_cast<size_t>(tid) * 66) : -INFINITY;
     const float lc = tid < nsplit ? __ldcg(src + static_cast<size_t>(tid) * 66 + 1) : 0.f;
+    float v[kMaxSplits];
+    const float* col = src + 2 + tid;
+#pragma unroll
+    for (int c = 0; c < kMaxSplits; ++c) v[c] = c < nsplit ? __ldcg(col + static_cast<size_t>(c) * 66) : 0.f;
     float M = mc;
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -453,11 +462,7 @@ __global__ void __launch_bounds__(64) global_rows_merge_kernel(const __grid_cons
     __syncthreads();
     L = red[0] + red[1];
 
-    // pass 2: column tid of every split, all loads first
-    float v[kMaxSplits];
-    const float* col = src + 2 + tid;
-#pragma unroll
-    for (int c = 0; c < kMaxSplits; ++c) v[c] = c < nsplit ? __ldcg(col + static_cast<size_t>(c) * 66) : 0.f;
+    // the weighted sum of the splits' columns
     float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
     for (int c = 0; c < kMaxSplits; c += 2) {

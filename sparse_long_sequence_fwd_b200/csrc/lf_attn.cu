@@ -66,7 +66,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int kMaxBandCtas = 296;
 
 struct Layout {
-    size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, off_bcnt, off_bpart, total;
+    size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, off_qg, off_bcnt, off_bpart,
+        total;
     int W, gstride, nchunk, ngp, cpc;  // nchunk: partial states per global row
     long long band_tiles;             // upper bound on the band kernel's tiles (its merge tickets)
 };
@@ -99,10 +100,12 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
     if (n_global > 0) o = align256(o + sizeof(float) * size_t(B) * H * L.gstride * L.nchunk * (d + 2));
     L.off_kg = o;
     L.off_vg = o;
+    L.off_qg = o;
     if (dtype == LF_BF16 && n_global > 0) {
         const size_t kgb = sizeof(__nv_bfloat16) * size_t(B) * H * L.ngp * 64;
         L.off_vg = align256(o + kgb);
-        o = align256(L.off_vg + kgb);
+        L.off_qg = align256(L.off_vg + kgb);
+        o = align256(L.off_qg + kgb);
     }
     L.off_bcnt = o;
     L.off_bpart = o;
@@ -126,7 +129,7 @@ bool is_capturing(cudaStream_t s) {
 // Shared-memory limits of every kernel, and the carveout that lets two band
 // CTAs share an SM.
 lf_status set_kernel_attributes() {
-    const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + kMaxGlobal) * 4;
+    const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + 2 * kMaxGlobal) * 4;
     const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
     if (cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) != cudaSuccess ||
         cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -346,6 +349,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
     ws.partial = reinterpret_cast<float*>(base + L.off_part);
     ws.kg = reinterpret_cast<__nv_bfloat16*>(base + L.off_kg);
     ws.vg = reinterpret_cast<__nv_bfloat16*>(base + L.off_vg);
+    ws.qg = reinterpret_cast<__nv_bfloat16*>(base + L.off_qg);
     const int r_eff = std::min(r, T);  // a window wider than the sequence changes nothing
     const float sl2 = static_cast<float>(double(scale) * kLog2e);
     int launches = 0;
@@ -354,6 +358,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
     PrepParams pp;
     pp.gidx = gidx;
     pp.pad = pad;
+    pp.q = q;
     pp.k = k;
     pp.v = v;
     pp.ws = ws;
@@ -366,7 +371,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
     pp.pack = (dtype == LF_BF16 && n_global > 0) ? 1 : 0;
     pp.band_cnt = reinterpret_cast<int32_t*>(base + L.off_bcnt);
     pp.n_band_cnt = static_cast<int>(L.band_tiles * 8);
-    const size_t prep_smem = size_t(L.W + 2 * kPrepThreads + L.gstride) * 4;
+    const size_t prep_smem = size_t(L.W + 2 * kPrepThreads + 2 * L.gstride) * 4;
     if (stages & 1u) {
         prep_kernel<<<B * H, kPrepThreads, prep_smem, stream>>>(pp);
         ++launches;
@@ -484,6 +489,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         gp.nchunk = L.nchunk;
         gp.sl2 = sl2;
         gp.cpc = L.cpc;
+        gp.ngp = L.ngp;
         if (dtype == LF_BF16) {
             // key splits x (b, h) x groups of 64 global rows, then the merge of the splits
             global_rows_mma_kernel<<<dim3(L.nchunk, B * H, (L.gstride + kGrRows - 1) / kGrRows), kGrWarps * 32,

@@ -29,6 +29,7 @@ struct Workspace {
     float* partial;     // [B*H][gstride][nchunk][d + 2] partial (m, l, acc) of each global row
     __nv_bfloat16* kg;  // [B*H][ngp][64] packed global keys (bf16 path)
     __nv_bfloat16* vg;  // [B*H][ngp][64] packed global values
+    __nv_bfloat16* qg;  // [B*H][ngp][64] packed global queries, in gq_list order, zero past n_gq
 };
 
 struct PrepParams {
@@ -36,12 +37,13 @@ struct PrepParams {
     int32_t* band_cnt;    // band kernel merge tickets, zeroed here (n_band_cnt entries)
     int n_band_cnt;
     const uint8_t* pad;   // [B][T] or null
+    const void* q;        // [B,H,T,d] (bf16 path: global query rows packed into qg)
     const void* k;        // [B,H,T,d] (bf16 path: packed into kg)
     const void* v;
     Workspace ws;
     uint32_t* status;
     int B, H, T, d, n_global, gstride, ngp, W;
-    int pack;             // 1: write kg/vg (bf16, d == 64)
+    int pack;             // 1: write kg/vg/qg (bf16, d == 64)
 };
 
 struct GlobalRowParams {
@@ -53,6 +55,7 @@ struct GlobalRowParams {
     Workspace ws;
     int B, H, T, d, gstride, nchunk;  // nchunk: partial states per global row
     int cpc;                          // bf16: 128-key chunks per CTA
+    int ngp;                          // bf16: rows per (b, h) of the packed global queries
     float sl2;  // scale * log2(e)
 };
 

@@ -13,7 +13,9 @@
 // uses for its (b, h), and (all CTAs together) the band kernel's merge
 // tickets.  On the bf16 path every CTA also packs the rows of k and v
 // named by gk_list into contiguous [ngp][64] blocks for its (b, h), zero
-// beyond the list, so the band kernel can stage them with one TMA box.
+// beyond the list, so the band kernel can stage them with one TMA box, and
+// the rows of q named by gq_list the same way, so the global-row kernel
+// reads its queries without first reading the list.
 #pragma once
 #include "lf_common.cuh"
 #include "ptx.cuh"
@@ -65,7 +67,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     int* scan_q = reinterpret_cast<int*>(bits + p.W);                // [256]
     int* scan_k = scan_q + kPrepThreads;                             // [256]
     int* gk_s = scan_k + kPrepThreads;                               // [gstride]
-    __shared__ int n_k_total;
+    int* gq_s = gk_s + p.gstride;                                    // [gstride]
+    __shared__ int n_k_total, n_q_total;
 
     grid_dep_launch();  // the band kernel may set itself up meanwhile; it waits for this grid before reading
     const int tid = threadIdx.x;
@@ -101,7 +104,10 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     }
     int oq = block_exclusive_scan(cq, scan_q);
     int ok = block_exclusive_scan(ck, scan_k);
-    if (tid == kPrepThreads - 1) n_k_total = ok + ck;
+    if (tid == kPrepThreads - 1) {
+        n_k_total = ok + ck;
+        n_q_total = oq + cq;
+    }
     const bool writer = (h == 0);
     int32_t* gq_out = p.ws.gq_list + static_cast<size_t>(b) * p.gstride;
     int32_t* gk_out = p.ws.gk_list + static_cast<size_t>(b) * p.gstride;
@@ -111,6 +117,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
         const uint32_t pw = (pad_b && qb) ? pad_word(pad_b, w, T) : 0u;
         for (uint32_t t = qb; t; t &= t - 1) {
             int j = (w << 5) + __ffs(t) - 1;
+            gq_s[oq] = j;
             if (writer) gq_out[oq] = j;
             ++oq;
             if (!((pw >> (j & 31)) & 1u)) {
@@ -127,22 +134,26 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     __syncthreads();
 
     if (p.pack) {
-        const int nk = n_k_total;
+        const int nk = n_k_total, nq = n_q_total;
         const size_t bh = static_cast<size_t>(b) * p.H + h;
+        const uint4* q4 = reinterpret_cast<const uint4*>(p.q) + bh * T * 8;
         const uint4* k4 = reinterpret_cast<const uint4*>(p.k) + bh * T * 8;
         const uint4* v4 = reinterpret_cast<const uint4*>(p.v) + bh * T * 8;
+        uint4* qg4 = reinterpret_cast<uint4*>(p.ws.qg) + bh * p.ngp * 8;
         uint4* kg4 = reinterpret_cast<uint4*>(p.ws.kg) + bh * p.ngp * 8;
         uint4* vg4 = reinterpret_cast<uint4*>(p.ws.vg) + bh * p.ngp * 8;
         for (int idx = tid; idx < p.ngp * 8; idx += kPrepThreads) {
             int a = idx >> 3, c = idx & 7;
-            uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+            uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv, qv = kv;
             if (a < nk) {
                 size_t row = static_cast<size_t>(gk_s[a]);
                 kv = k4[row * 8 + c];
                 vv = v4[row * 8 + c];
             }
+            if (a < nq) qv = q4[static_cast<size_t>(gq_s[a]) * 8 + c];
             kg4[idx] = kv;
             vg4[idx] = vv;
+            qg4[idx] = qv;
         }
     }
 }
