@@ -189,28 +189,41 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
 
 
 // bf16, d = 64: tensor-core global rows.  CTA (split, b*h, row group) takes
-// up to 64 global queries of sample b (16 per warp: one m16n8k16 row tile)
-// and cpc consecutive 128-key chunks of the key axis.  The chunks of K and V
-// stream through a two-stage ring in padded shared memory (cp.async,
-// zero-filled past T); the first two are requested before anything that
-// depends on the prep kernel (the global-query count and the query rows,
-// which prep packs in list order), so the HBM latency overlaps those reads.  Every warp forms
-// S = Q K^T (16 x 128, fp32 in registers), applies the key padding mask,
-// runs the online softmax (log2 domain, exp2) and accumulates O += P V with
-// P re-packed from the S registers as bf16 A fragments and V fragments from
-// ldmatrix.trans.  The partial state (m, l, O) of each row and split goes to
-// the workspace; global_rows_merge_kernel combines the splits.  This path is
-// bound by HBM traffic (every K/V row of a (b, h) is read once per row
-// group), not by the tensor rate, so the synchronous warp-level MMA is
-// enough.
+// up to KPW / 2 global queries of sample b and cpc consecutive 128-key
+// chunks of the key axis.  Its 4 warps form an RG x KP grid: RG row tiles of
+// 16 queries (one m16n8k16 row tile each) times KP key slices of KPW keys,
+// warp (rg, kp) taking keys [kp KPW, (kp + 1) KPW) of every chunk for the
+// queries of row tile rg.  With few global queries the warps split the keys
+// instead of idling, so all four SM sub-partitions run the warp-level MMA.
+// The chunks of K and V stream through a two-stage ring in padded shared
+// memory (cp.async, zero-filled past T); the first two are requested before
+// anything that depends on the prep kernel (the global-query count and the
+// query rows, which prep packs in list order), so the HBM latency overlaps
+// those reads.  Every warp forms S = Q K^T (16 x KPW, fp32 in registers),
+// applies the key padding mask, runs the online softmax (log2 domain, exp2)
+// and accumulates O += P V with P re-packed from the S registers as bf16 A
+// fragments and V fragments from ldmatrix.trans.  At the end the KP slices of
+// a row tile combine their states (m, l, O) through shared memory in slice
+// order, and the result goes to the workspace as this split's partial state;
+// global_rows_merge_kernel combines the splits.  Every K/V row of a (b, h) is
+// read once per row group; the warp-level MMA (a quarter of the tcgen05
+// rate) keeps up with that as long as every sub-partition issues it.
 constexpr int kGrKeys = 128;       // keys per chunk
-constexpr int kGrWarps = 4;        // 16 rows per warp
-constexpr int kGrRows = 16 * kGrWarps;
+constexpr int kGrWarps = 4;        // row tiles x key slices
+constexpr int kGrXchFloats = 36;   // per lane when slices combine: m_a, m_b, l_a, l_b, O[8][4]
+// Keys per warp slice of a chunk for a global-query capacity: every warp
+// gets work whatever the count (16 queries or fewer: 4 slices of 32 keys;
+// 32 or fewer: 2 row tiles x 2 slices of 64; more: 4 row tiles x 128 keys).
+// A CTA then holds KPW / 2 global-query slots.  (The host takes 128, no
+// slices, when every CTA has a single chunk: the combine would cost more
+// than the slices save.)
+__host__ __device__ constexpr int gr_kpw(int gstride) { return gstride <= 16 ? 32 : (gstride <= 32 ? 64 : 128); }
 constexpr int kGrStride = 72;      // bf16 per staged row: 64 + 8 (conflict-free fragments and ldmatrix)
 constexpr int kGrStages = 2;
 constexpr int kGrChunkElems = kGrKeys * kGrStride;          // bf16 per K (or V) chunk
 constexpr int kGrSmem = kGrStages * 2 * kGrChunkElems * 2;  // bytes of the ring
 constexpr int kMaxSplits = 64;                              // key splits per (b, h): the merge holds them in registers
+static_assert(kGrWarps * kGrXchFloats * 32 * 4 <= kGrSmem, "slice states fit in the ring");
 
 __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -234,12 +247,21 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+template <int KPW>
 __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const __grid_constant__ GlobalRowParams p) {
+    constexpr int KP = kGrKeys / KPW;    // key slices of a chunk
+    constexpr int RG = kGrWarps / KP;    // row tiles of 16 queries
+    constexpr int ROWS = 16 * RG;        // global-query slots per CTA
+    constexpr int NT = KPW / 8;          // 8-key tiles of a slice (S columns)
+    constexpr int KK = KPW / 16;         // 16-key steps of a slice (P V)
+    static_assert(KP * RG == kGrWarps, "the warps cover row tiles x slices");
     extern __shared__ __align__(16) __nv_bfloat16 gr_ring[];  // [stage][K, V][kGrKeys][kGrStride]
     __shared__ uint32_t valid_bits[kGrStages][kGrKeys / 32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g8 = lane >> 2, t4 = lane & 3;  // fragment row group and column pair
+    const int rg = warp % RG, kp = warp / RG;
+    const int k0 = kp * KPW;                  // this warp's first key in every chunk
     const int split = blockIdx.x, bh = blockIdx.y, b = bh / p.H;
     const int T = p.T;
     const size_t base = static_cast<size_t>(bh) * T * 64;
@@ -269,7 +291,7 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
     // Q fragments of rows row0 + g8 and row0 + g8 + 8 from the packed global
     // queries (prep's output: zero past the sample's count, so no count or list
     // is needed first), loaded alongside the count
-    const int row0 = blockIdx.z * kGrRows + warp * 16;  // this warp's first global-row slot
+    const int row0 = blockIdx.z * ROWS + rg * 16;  // this warp's first global-row slot
     uint32_t qa[4][4];
     {
         const __nv_bfloat16* qgb = p.ws.qg + static_cast<size_t>(bh) * p.ngp * 64;
@@ -286,7 +308,7 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
         }
     }
     const int nq = p.ws.n_gq[b];
-    if (blockIdx.z * kGrRows >= nq) {
+    if (blockIdx.z * ROWS >= nq) {
         cp_async_wait<0>();  // no copy may still target this CTA's shared memory
         return;
     }
@@ -314,12 +336,12 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
         cp_async_wait<1>();  // this chunk has landed (the next one may still be in flight)
         __syncthreads();
         if (active) {
-            // S = Q K^T: 16 key tiles of 8
-            float s[16][4];
+            // S = Q K^T over this warp's slice: NT key tiles of 8
+            float s[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
+            for (int nt = 0; nt < NT; ++nt) {
                 s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-                const __nv_bfloat16* kr = Ks + (8 * nt + g8) * kGrStride + 2 * t4;
+                const __nv_bfloat16* kr = Ks + (k0 + 8 * nt + g8) * kGrStride + 2 * t4;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks);
@@ -327,11 +349,12 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
                     mma_bf16_16816(s[nt], qa[ks], b0, b1);
                 }
             }
-            // mask, scale, row maxima (each row's 128 scores live in the 4 lanes of its quad)
+            // mask, scale, row maxima (each row's scores live in the 4 lanes of its quad)
             float mx_a = -INFINITY, mx_b = -INFINITY;
 #pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                const uint32_t vw = valid_bits[st][nt >> 2] >> ((nt & 3) * 8 + 2 * t4);
+            for (int nt = 0; nt < NT; ++nt) {
+                const int key = k0 + 8 * nt;  // first key of the tile; this lane has key + 2 t4, + 1
+                const uint32_t vw = valid_bits[st][key >> 5] >> ((key & 31) + 2 * t4);
                 const bool v0 = vw & 1u, v1 = (vw >> 1) & 1u;
                 s[nt][0] = v0 ? s[nt][0] * sl2 : -INFINITY;
                 s[nt][1] = v1 ? s[nt][1] * sl2 : -INFINITY;
@@ -361,9 +384,9 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
                 o[nd][3] *= al_b;
             }
             // P (bf16 A fragments) and row sums
-            uint32_t pa[8][4];
+            uint32_t pa[KK][4];
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
+            for (int kk = 0; kk < KK; ++kk) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     float* sv = s[2 * kk + h];
@@ -377,12 +400,12 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
             }
             // O += P V: for each 16-key step, two 8-column tiles of V per ldmatrix
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
+            for (int kk = 0; kk < KK; ++kk) {
                 const uint32_t a4[4] = {pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3]};
 #pragma unroll
                 for (int nd = 0; nd < 8; nd += 2) {
                     uint32_t vf[4];
-                    ldmatrix_x4_trans(vf, Vs + (16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1)) * kGrStride +
+                    ldmatrix_x4_trans(vf, Vs + (k0 + 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1)) * kGrStride +
                                               8 * (nd + (lane >> 4)));
                     mma_bf16_16816(o[nd], a4, vf[0], vf[1]);
                     mma_bf16_16816(o[nd + 1], a4, vf[2], vf[3]);
@@ -394,13 +417,64 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
         cp_async_commit();  // (empty past the last chunk, so every wait above counts the same)
     }
     cp_async_wait<0>();
-    if (!active) return;
-    // full row sums over the quad, then the partial state of each row
+    // full row sums over the quad
 #pragma unroll
     for (int off = 1; off <= 2; off <<= 1) {
         l_a += __shfl_xor_sync(0xffffffffu, l_a, off);
         l_b += __shfl_xor_sync(0xffffffffu, l_b, off);
     }
+    if (KP > 1) {
+        // the slices' states through shared memory (the ring is free: every copy
+        // has landed and been consumed), then the first slice of each row tile
+        // combines them in slice order: M = max m_k, w_k = 2^(m_k - M),
+        // L = sum w_k l_k, O = sum w_k O_k
+        __syncthreads();
+        float* xs = reinterpret_cast<float*>(gr_ring);  // [warp][kGrXchFloats][32 lanes]
+        {
+            float* mine = xs + warp * kGrXchFloats * 32 + lane;
+            mine[0] = m_a;
+            mine[32] = m_b;
+            mine[64] = l_a;
+            mine[96] = l_b;
+#pragma unroll
+            for (int nd = 0; nd < 8; ++nd)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) mine[(4 + 4 * nd + j) * 32] = o[nd][j];
+        }
+        __syncthreads();
+        if (kp != 0 || !active) return;
+        float Ma = -INFINITY, Mb = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < KP; ++q) {
+            const float* src = xs + (q * RG + rg) * kGrXchFloats * 32 + lane;
+            Ma = fmaxf(Ma, src[0]);
+            Mb = fmaxf(Mb, src[32]);
+        }
+        const float Mua = Ma == -INFINITY ? 0.f : Ma, Mub = Mb == -INFINITY ? 0.f : Mb;
+        l_a = l_b = 0.f;
+#pragma unroll
+        for (int nd = 0; nd < 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+#pragma unroll
+        for (int q = 0; q < KP; ++q) {
+            const float* src = xs + (q * RG + rg) * kGrXchFloats * 32 + lane;
+            const float wa = src[0] == -INFINITY ? 0.f : ex2_approx(src[0] - Mua);
+            const float wb = src[32] == -INFINITY ? 0.f : ex2_approx(src[32] - Mub);
+            l_a = fmaf(wa, src[64], l_a);
+            l_b = fmaf(wb, src[96], l_b);
+#pragma unroll
+            for (int nd = 0; nd < 8; ++nd) {
+                o[nd][0] = fmaf(wa, src[(4 + 4 * nd) * 32], o[nd][0]);
+                o[nd][1] = fmaf(wa, src[(5 + 4 * nd) * 32], o[nd][1]);
+                o[nd][2] = fmaf(wb, src[(6 + 4 * nd) * 32], o[nd][2]);
+                o[nd][3] = fmaf(wb, src[(7 + 4 * nd) * 32], o[nd][3]);
+            }
+        }
+        m_a = Ma;
+        m_b = Mb;
+    } else if (!active) {
+        return;
+    }
+    // the partial state of each row of this split
     const int nsplit = p.nchunk;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {

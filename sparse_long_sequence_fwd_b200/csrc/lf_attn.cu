@@ -69,6 +69,7 @@ struct Layout {
     size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, off_qg, off_bcnt, off_bpart,
         total;
     int W, gstride, nchunk, ngp, cpc;  // nchunk: partial states per global row
+    int gr_kpw;                        // bf16 global rows: keys per warp slice of a chunk
     long long band_tiles;             // upper bound on the band kernel's tiles (its merge tickets)
 };
 
@@ -80,8 +81,19 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
         // tensor-core global rows: 128-key chunks, cpc per CTA, about three CTAs
         // per SM of a 148-SM B200 (each holds a two-stage ring of 72 KB)
         const int nblk = (T + kGrKeys - 1) / kGrKeys;
-        const long units = long(nblk) * B * H * ((L.gstride + kGrRows - 1) / kGrRows);
-        L.cpc = static_cast<int>(std::max(1L, std::min<long>(nblk, (units + 443) / 444)));
+        // Warps split each chunk's keys when there are few global queries, but
+        // combining the slices only pays off when a CTA takes two chunks or more.
+        auto chunks_per_cta = [&](int kpw) {
+            const int rows = kpw / 2;  // global-query slots per CTA
+            const long units = long(nblk) * B * H * ((L.gstride + rows - 1) / rows);
+            return static_cast<int>(std::max(1L, std::min<long>(nblk, (units + 443) / 444)));
+        };
+        L.gr_kpw = gr_kpw(L.gstride);
+        L.cpc = chunks_per_cta(L.gr_kpw);
+        if (L.cpc == 1 && L.gr_kpw != kGrKeys) {
+            L.gr_kpw = kGrKeys;
+            L.cpc = chunks_per_cta(L.gr_kpw);
+        }
         L.nchunk = (nblk + L.cpc - 1) / L.cpc;
         while (L.nchunk > kMaxSplits) L.nchunk = (nblk + ++L.cpc - 1) / L.cpc;
     } else {
@@ -141,7 +153,12 @@ lf_status set_kernel_attributes() {
             cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(global_rows_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) != cudaSuccess)
+        cudaFuncSetAttribute(global_rows_mma_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) !=
+            cudaSuccess)
         return LF_ERR_CUDA;
     return LF_OK;
 }
@@ -491,9 +508,12 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         gp.cpc = L.cpc;
         gp.ngp = L.ngp;
         if (dtype == LF_BF16) {
-            // key splits x (b, h) x groups of 64 global rows, then the merge of the splits
-            global_rows_mma_kernel<<<dim3(L.nchunk, B * H, (L.gstride + kGrRows - 1) / kGrRows), kGrWarps * 32,
-                                     kGrSmem, gs>>>(gp);
+            // key splits x (b, h) x groups of kpw / 2 global rows, then the merge of the splits
+            const int kpw = L.gr_kpw, rows = kpw / 2;
+            const dim3 grid(L.nchunk, B * H, (L.gstride + rows - 1) / rows);
+            if (kpw == 32) global_rows_mma_kernel<32><<<grid, kGrWarps * 32, kGrSmem, gs>>>(gp);
+            else if (kpw == 64) global_rows_mma_kernel<64><<<grid, kGrWarps * 32, kGrSmem, gs>>>(gp);
+            else global_rows_mma_kernel<128><<<grid, kGrWarps * 32, kGrSmem, gs>>>(gp);
             // the merge is the split kernel's programmatic dependent: it launches while the
             // splits finish and waits for them (griddepcontrol.wait) before reading
             cudaLaunchConfig_t mc = {};

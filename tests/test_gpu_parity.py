@@ -186,6 +186,18 @@ def test_split_piece_then_one_block_split_piece(dil, n_random):
     parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
 
 
+@pytest.mark.parametrize("n_random,pad", [(9, 3900), (27, None)])
+def test_global_rows_split_keys_between_warps(n_random, pad):
+    """With 16 or fewer global queries (or 17 to 32) and two 128-key chunks per
+    CTA of the global-row kernel (16 heads x 32 chunks > one wave), its warps
+    split each chunk's keys into 4 (or 2) slices and combine them at the end;
+    every element is compared with the oracle, padding included."""
+    w = workloads.custom("gr_slices_%d" % n_random, "bf16", 1, 16, 4096, 64, 40, n_random_globals=n_random,
+                         pad_from=[pad], seed=46)
+    inp = workloads.make_inputs(w)
+    parity.compare(w, parity.run_gpu(w, inp), parity.oracle_full(w, inp))
+
+
 def test_out_of_range_global_entries_are_ignored_and_flagged():
     w = workloads.custom("bad_g", "bf16", 1, 2, 300, 64, 20, seed=40)
     inp = workloads.make_inputs(w)
