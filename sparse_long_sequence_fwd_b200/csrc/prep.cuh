@@ -96,11 +96,25 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     const int per = (p.W + kPrepThreads - 1) / kPrepThreads;
     const int w0 = min(p.W, tid * per), w1 = min(p.W, w0 + per);
     int cq = 0, ck = 0;
+    // padding words of this thread's words that hold global tokens, kept for the
+    // second pass (each costs 32 byte loads); two cover T <= 16384
+    int pw_w[2] = {-1, -1};
+    uint32_t pw_v[2] = {0u, 0u};
     for (int w = w0; w < w1; ++w) {
         uint32_t qb = bits[w];
         cq += __popc(qb);
-        const uint32_t kb = (pad_b && qb) ? (qb & ~pad_word(pad_b, w, T)) : qb;
-        ck += __popc(kb);
+        uint32_t pw = 0u;
+        if (pad_b && qb) {
+            pw = pad_word(pad_b, w, T);
+            if (pw_w[0] < 0) {
+                pw_w[0] = w;
+                pw_v[0] = pw;
+            } else if (pw_w[1] < 0) {
+                pw_w[1] = w;
+                pw_v[1] = pw;
+            }
+        }
+        ck += __popc(qb & ~pw);
     }
     int oq = block_exclusive_scan(cq, scan_q);
     int ok = block_exclusive_scan(ck, scan_k);
@@ -114,7 +128,10 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     for (int w = w0; w < w1; ++w) {
         uint32_t qb = bits[w];
         if (writer) p.ws.gbit[static_cast<size_t>(b) * p.W + w] = qb;
-        const uint32_t pw = (pad_b && qb) ? pad_word(pad_b, w, T) : 0u;
+        const uint32_t pw = !(pad_b && qb) ? 0u
+                            : w == pw_w[0]   ? pw_v[0]
+                            : w == pw_w[1]   ? pw_v[1]
+                                             : pad_word(pad_b, w, T);
         for (uint32_t t = qb; t; t &= t - 1) {
             int j = (w << 5) + __ffs(t) - 1;
             gq_s[oq] = j;
@@ -142,7 +159,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
         uint4* qg4 = reinterpret_cast<uint4*>(p.ws.qg) + bh * p.ngp * 8;
         uint4* kg4 = reinterpret_cast<uint4*>(p.ws.kg) + bh * p.ngp * 8;
         uint4* vg4 = reinterpret_cast<uint4*>(p.ws.vg) + bh * p.ngp * 8;
-        for (int idx = tid; idx < p.ngp * 8; idx += kPrepThreads) {
+#pragma unroll 4
+        for (int idx = tid; idx < p.ngp * 8; idx += kPrepThreads) {  // (unrolled: the loads of several rows in flight)
             int a = idx >> 3, c = idx & 7;
             uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv, qv = kv;
             if (a < nk) {
