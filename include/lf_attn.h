@@ -95,7 +95,7 @@ lf_status lf_attn_fwd(const void* q, const void* k, const void* v, void* out,
  * layouts above (page-locked memory gives full copy bandwidth).  The call
  * copies the inputs into a library-owned device staging area, runs the
  * forward and copies `out` back, ordered after the work already queued on
- * `stream`, and returns when `out` is ready.  It works on up to 8 slices
+ * `stream`, and returns when `out` is ready.  It works on up to 4 slices
  * of (sample, group of heads): the inputs of a slice are copied on a
  * library-owned copy-in stream, its kernels run on `stream`, and its output
  * is copied back on a copy-out stream, so the copies of one slice overlap
