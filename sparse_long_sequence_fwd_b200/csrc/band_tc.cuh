@@ -723,6 +723,9 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
     }
 }
 
+// kSearch: the sample may have more than 32 global keys; the global-key block's
+// dedup then finds the keys in a row's window by binary search (below).
+template <bool kSearch>
 __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                              volatile int* abort_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -848,6 +851,38 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                         }
                         const int gb = blk - nbb;
                         const int nvalid = min(kBN, ngk - gb * kBN);
+                        bool searched = false;
+                        if constexpr (kSearch) {
+                            if (ngk <= kBN) {
+                                // all the keys are in registers, sorted and unique: the ones in
+                                // this row's window are the index range [lo, hi) of the keys in
+                                // [i - dil r, i + dil r] (two binary searches), within the row's
+                                // residue class (the same for every row of the tile)
+                                const int reach_s = dp->dil * p.r;
+                                auto count_below = [&](int t) -> int {  // keys < t
+                                    int pos = 0;
+#pragma unroll
+                                    for (int step = 64; step >= 1; step >>= 1) {
+                                        const int probe = min(pos + step - 1, kBN - 1);
+                                        const int k0 = static_cast<int>(__shfl_sync(0xffffffffu, gk_reg[0], probe & 31));
+                                        const int k1 = static_cast<int>(__shfl_sync(0xffffffffu, gk_reg[1], probe & 31));
+                                        if (pos + step - 1 < ngk && (probe < 32 ? k0 : k1) < t) pos += step;
+                                    }
+                                    return pos;
+                                };
+                                const int lo = count_below(i - reach_s), hi = count_below(i + reach_s + 1);
+#pragma unroll
+                                for (int c = 0; c < 2; ++c) {
+                                    uint32_t in_win = range_bits(lo - 32 * c, hi - 32 * c);
+                                    if (dp->dil > 1)
+                                        in_win &= __ballot_sync(0xffffffffu,
+                                                                static_cast<int>(gk_reg[c]) % dp->dil == dp->c);
+                                    mk[c] = range_bits(0, nvalid - 32 * c) & ~in_win;
+                                }
+                                searched = true;
+                            }
+                        }
+                        if (!searched) {
                         const int32_t* gkl = p.gk_list + static_cast<size_t>(bs) * p.gstride + gb * kBN;
                         const int dil = dp->dil, reach = dil * p.r;
 #pragma unroll
@@ -864,6 +899,7 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                                 }
                             }
                             mk[c] = m;
+                        }
                         }
                     }
                     live0 = __any_sync(0xffffffffu, mk[0] != 0u);
@@ -972,6 +1008,10 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     }
 }
 
+// Two instantiations from one source: kSearch = true for calls with more than
+// 32 global tokens (see softmax_role), false otherwise, so each keeps its own
+// code for the block loop.
+template <bool kSearch>
 __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(const __grid_constant__ BandTcParams p) {
     extern __shared__ uint8_t band_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(band_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1039,7 +1079,7 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
                 asm volatile("" ::"r"(v));
             }
         }
-        softmax_role(p, smem, bars, abort_flag, tmem_base);
+        softmax_role<kSearch>(p, smem, bars, abort_flag, tmem_base);
     }
 
     tc_fence_before();

@@ -145,8 +145,13 @@ bool is_capturing(cudaStream_t s) {
 lf_status set_kernel_attributes() {
     const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + 2 * kMaxGlobal) * 4;
     const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
-    if (cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(band_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+    if (cudaFuncSetAttribute(band_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(band_tc_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaFuncSetAttribute(band_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(band_tc_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
         cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) != cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
@@ -485,7 +490,9 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         attr[0].val.programmaticStreamSerializationAllowed = (stages & 1u) ? 1 : 0;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, band_tc_kernel, bp) != cudaSuccess) return LF_ERR_CUDA;
+        // more than 32 global tokens: the instantiation whose global-key dedup searches
+        if (cudaLaunchKernelEx(&cfg, n_global > 32 ? band_tc_kernel<true> : band_tc_kernel<false>, bp) != cudaSuccess)
+            return LF_ERR_CUDA;
         ++launches;
     }
 

@@ -48,6 +48,10 @@ SMALL = [
                      globals_per_b=[[0]], seed=12),
     workloads.custom("bf16_many_globals", "bf16", 1, 2, 1200, 64, 64, dil=[1, 4],
                      globals_per_b=[list(range(0, 1200, 4))], pad_from=[1100], seed=13),
+    # 33 to 64 distinct global tokens (duplicates in the list), dilated heads, padding
+    workloads.custom("bf16_49_globals_dil", "bf16", 2, 4, 1500, 64, 60, dil=[1, 2, 3, 4],
+                     globals_per_b=[list(range(5, 1500, 31)) + [5, 36], list(range(700, 1100, 9)) + [1096] * 6],
+                     pad_from=[1400, None], seed=18),
     workloads.custom("bf16_dil_5_to_8", "bf16", 1, 4, 700, 64, 20, dil=[5, 6, 7, 8],
                      globals_per_b=[[1, 2, 699]], seed=14),
     workloads.custom("f32_multi_tile", "f32", 2, 3, 600, 64, 70, dil=[1, 2, 3],
