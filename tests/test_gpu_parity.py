@@ -52,6 +52,9 @@ SMALL = [
     workloads.custom("bf16_49_globals_dil", "bf16", 2, 4, 1500, 64, 60, dil=[1, 2, 3, 4],
                      globals_per_b=[list(range(5, 1500, 31)) + [5, 36], list(range(700, 1100, 9)) + [1096] * 6],
                      pad_from=[1400, None], seed=18),
+    # 3 global rows over 64 key splits
+    workloads.custom("bf16_64_splits_3_globals", "bf16", 1, 2, 16384, 64, 32,
+                     globals_per_b=[[5, 16000, 9000]], pad_from=[15000], seed=19),
     workloads.custom("bf16_dil_5_to_8", "bf16", 1, 4, 700, 64, 20, dil=[5, 6, 7, 8],
                      globals_per_b=[[1, 2, 699]], seed=14),
     workloads.custom("f32_multi_tile", "f32", 2, 3, 600, 64, 70, dil=[1, 2, 3],
@@ -218,12 +221,12 @@ def test_out_of_range_global_entries_are_ignored_and_flagged():
     assert st == 0 and flags == 0
 
 
-def test_deterministic_and_four_launches():
+@pytest.mark.parametrize("w,launches", [(workloads.BASE, 4), (workloads.QA, 4)], ids=["1_global", "64_globals"])
+def test_deterministic_and_launch_count(w, launches):
     """prep, band, global rows, merge of the global rows' key splits."""
-    w = workloads.BASE
     inp = workloads.make_inputs(w)
     a = parity.run_gpu(w, inp)
-    assert lf_attn.last_launch_count() == 4
+    assert lf_attn.last_launch_count() == launches
     b = parity.run_gpu(w, inp)
     assert torch.equal(a, b)
 
