@@ -58,7 +58,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
-    ap.add_argument("--no-others", action="store_true", help="skip the QA, dilated and large workload entries")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the QA, dilated, large and f16 base workload entries")
     return ap.parse_args()
 
 
@@ -204,7 +205,7 @@ class WorkloadRun:
         self.total_f, self.band_f, self.gr_f, self.gr_bytes = split_flops(w, inp)
         props = torch.cuda.get_device_properties(dev)
         self.l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
-        es = 2 if w.dtype == "bf16" else 4
+        es = 4 if w.dtype == "f32" else 2
         self.set_bytes = 4 * w.B * w.H * w.T * w.d * es
         self.n_sets = max(2, math.ceil(2 * self.l2 / self.set_bytes) + 1)
         q0, k0, v0 = (inp[x].to(dev) for x in ("q", "k", "v"))
@@ -394,7 +395,7 @@ def run_ours(args):
     # ---- the other workloads (each its own rotating inputs), rank 0 only
     others = {}
     if rank == 0 and world == 1 and not args.no_others:
-        for name in ("qa_B2_T4096_g64_pad", "dilated_T8192_r128", "large_T16384_g32"):
+        for name in ("qa_B2_T4096_g64_pad", "dilated_T8192_r128", "large_T16384_g32", "base_T4096_w513_f16"):
             if name == w.name:
                 continue
             ow = workloads.BY_NAME[name]

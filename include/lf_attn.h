@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-typedef enum { LF_F32 = 0, LF_BF16 = 1 } lf_dtype;
+typedef enum { LF_F32 = 0, LF_BF16 = 1, LF_F16 = 2 } lf_dtype;
 
 typedef enum {
     LF_OK = 0,
@@ -73,6 +73,10 @@ typedef enum {
  *               LF_BF16: tensor-core path (tcgen05 + TMA), d == 64 only,
  *               fp32 accumulation and softmax, every dil[h] <= 8, at most 4
  *               distinct dilation values, H <= 128.
+ *               LF_F16: the same tensor-core path with fp16 q, k, v and out
+ *               (fp16 MMA operands, the probabilities rounded to fp16 for the
+ *               P V product), with the same limits.  The pages train with
+ *               fp16 mixed precision (Longformer wiki, section 6.3).
  *   stream      a cudaStream_t (NULL = legacy default stream)
  *
  * Returns LF_OK once the kernels are queued; nothing is synchronised.

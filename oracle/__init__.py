@@ -57,7 +57,7 @@ def _load():
 
 
 def _f32(x) -> np.ndarray:
-    if hasattr(x, "detach"):  # torch tensor (fp32 or bf16): bf16 widens exactly to fp32
+    if hasattr(x, "detach"):  # torch tensor (fp32, bf16 or f16): the 16-bit types widen exactly to fp32
         import torch
         x = x.detach().to("cpu", torch.float32).numpy()
     return np.ascontiguousarray(x, dtype=np.float32)

@@ -419,9 +419,11 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
 // O += P(g-1) V(g-1) once P(g-1) is in TMEM.  Every product commits to the
 // O-complete barrier of its parity (two barriers, so a softmax thread that
 // only sometimes waits for a product can still tell the phases apart).
+// kHalf: q, k, v (and so P) are f16 instead of bf16.
+template <bool kHalf>
 __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                          volatile int* abort_flag, uint32_t tmem_base) {
-    const uint32_t idesc_pv = idesc_bf16(kBM, kHD, 0, 1);
+    const uint32_t idesc_pv = kHalf ? idesc_f16(kBM, kHD, 0, 1) : idesc_bf16(kBM, kHD, 0, 1);
     uint64_t dQ[kQStages];
 #pragma unroll
     for (int st = 0; st < kQStages; ++st) dQ[st] = sdesc_k_sw128(smem_u32(smem + kOffQ + st * kQBytes));
@@ -475,7 +477,7 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
                 ngk = *reinterpret_cast<const volatile int*>(p.n_gk + bsm);
             }
             const int ncols = blk < nbb ? kBN : global_block_cols(ngk, blk - nbb);
-            const uint32_t ids = idesc_bf16(kBM, ncols, 0, 0);
+            const uint32_t ids = kHalf ? idesc_f16(kBM, ncols, 0, 0) : idesc_bf16(kBM, ncols, 0, 0);
             const uint64_t dq = dQ[qs], dk = dK0 + kKVDescStep * st;
             const uint32_t tS = tmem_base + 64u * b;
             tc_mma<false>(tS, dq + 0, dk + 0, ids);  // K-steps of 16 (32 bytes = 2 units)
@@ -526,6 +528,7 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 // with two rounds of xor shuffles, after which store e of lane 4g + j writes
 // chunk j of row 4g + e.  (One lane per row would make every store touch 32
 // lines.)  Warp-wide: every lane calls it.
+template <bool kHalf>
 __device__ __forceinline__ void store_half_rows(__nv_bfloat16* row_ptr, bool write, int hd, const float* o,
                                                 float inv) {
     const int lane = threadIdx.x & 31;
@@ -533,7 +536,7 @@ __device__ __forceinline__ void store_half_rows(__nv_bfloat16* row_ptr, bool wri
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int w = 0; w < 4; ++w) x[c][w] = pack_bf16x2(o[8 * c + 2 * w] * inv, o[8 * c + 2 * w + 1] * inv);
+        for (int w = 0; w < 4; ++w) x[c][w] = pack16x2<kHalf>(o[8 * c + 2 * w] * inv, o[8 * c + 2 * w + 1] * inv);
 #pragma unroll
     for (int sh = 2; sh >= 1; sh >>= 1) {
         const bool upper = (lane & sh) != 0;
@@ -572,6 +575,7 @@ __device__ __forceinline__ float* part_slot(const BandTcParams& p, int s, int ts
 // descriptor d stays in shared memory until this is done; m and l are this
 // thread's row's exponent base and sum.  The row is handled 32 output
 // dimensions at a time (registers: this runs with the next piece's state live).
+template <bool kHalf>
 __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiece* d, float m, float l, uint32_t tO,
                                           int wq, int ticket, volatile int* abort_flag) {
     const int lane = threadIdx.x & 31;
@@ -596,7 +600,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
         for (int hd = 0; hd < 2; ++hd) {
             float o[32];
             load_o(hd, o);
-            store_half_rows(dst, write, hd, o, inv);
+            store_half_rows<kHalf>(dst, write, hd, o, inv);
         }
         return;
     }
@@ -667,7 +671,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
                     o[4 * u + k] = fmaf(w2, self_first ? a[k] : b, w1 * (self_first ? b : a[k]));
                 }
             }
-            store_half_rows(dst, write, hd, o, inv);
+            store_half_rows<kHalf>(dst, write, hd, o, inv);
         }
     } else {
         float M = m;
@@ -713,7 +717,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
                     acc[4 * u + 3] = fmaf(wv, v.w, acc[4 * u + 3]);
                 }
             }
-            store_half_rows(dst, write, hd, acc, inv);
+            store_half_rows<kHalf>(dst, write, hd, acc, inv);
         }
     }
     __syncwarp();
@@ -725,7 +729,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
 
 // kSearch: the sample may have more than 32 global keys; the global-key block's
 // dedup then finds the keys in a row's window by binary search (below).
-template <bool kSearch>
+template <bool kSearch, bool kHalf>
 __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                              volatile int* abort_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -776,7 +780,7 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     int ticket_prev = 0;  // the previous piece's, kept until its rows are written
     auto finish_prev = [&]() {
         const BandPiece* dq = reinterpret_cast<const BandPiece*>(smem + kOffDesc + prev_slot * kDescBytes);
-        flush_rows(p, dq, m_prev, l_prev, tO, wq, __shfl_sync(0xffffffffu, ticket_prev, 0), abort_flag);
+        flush_rows<kHalf>(p, dq, m_prev, l_prev, tO, wq, __shfl_sync(0xffffffffu, ticket_prev, 0), abort_flag);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarQEmpty + prev_slot]);
         prev_slot = -1;
@@ -966,8 +970,8 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                             const float2 e1 = make_float2(ex2_approx(t1.x), ex2_approx(t1.y));
                             acc0 = fadd2(acc0, e0);
                             acc1 = fadd2(acc1, e1);
-                            pk[16 * c + j / 2] = pack_bf16x2(e0.x, e0.y);
-                            pk[16 * c + j / 2 + 1] = pack_bf16x2(e1.x, e1.y);
+                            pk[16 * c + j / 2] = pack16x2<kHalf>(e0.x, e0.y);
+                            pk[16 * c + j / 2 + 1] = pack16x2<kHalf>(e1.x, e1.y);
                         }
                     } else {
 #pragma unroll
@@ -1008,10 +1012,10 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     }
 }
 
-// Two instantiations from one source: kSearch = true for calls with more than
-// 32 global tokens (see softmax_role), false otherwise, so each keeps its own
-// code for the block loop.
-template <bool kSearch>
+// Instantiations from one source: kSearch = true for calls with more than 32
+// global tokens (see softmax_role), false otherwise, so each keeps its own
+// code for the block loop; kHalf = true for f16 inputs, false for bf16.
+template <bool kSearch, bool kHalf>
 __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(const __grid_constant__ BandTcParams p) {
     extern __shared__ uint8_t band_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(band_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1068,7 +1072,7 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
     if (warp == 0) {
         if (lane == 0) producer_role(p, smem, bars, abort_flag);
     } else if (warp == 1) {
-        if (lane == 0) mma_role(p, smem, bars, abort_flag, tmem_base);
+        if (lane == 0) mma_role<kHalf>(p, smem, bars, abort_flag, tmem_base);
     } else {
         {  // touch every 64-byte line of the parameters once, so the producer's walk hits in cache
             const int t = threadIdx.x - 64;
@@ -1079,7 +1083,7 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
                 asm volatile("" ::"r"(v));
             }
         }
-        softmax_role<kSearch>(p, smem, bars, abort_flag, tmem_base);
+        softmax_role<kSearch, kHalf>(p, smem, bars, abort_flag, tmem_base);
     }
 
     tc_fence_before();

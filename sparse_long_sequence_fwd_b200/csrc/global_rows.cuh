@@ -225,12 +225,21 @@ constexpr int kGrSmem = kGrStages * 2 * kGrChunkElems * 2;  // bytes of the ring
 constexpr int kMaxSplits = 64;                              // key splits per (b, h): the merge holds them in registers
 static_assert(kGrWarps * kGrXchFloats * 32 * 4 <= kGrSmem, "slice states fit in the ring");
 
-__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// D += A B, m16n8k16, fp32 accumulators; A and B bf16 (kHalf: f16).
+template <bool kHalf>
+__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    if constexpr (kHalf)
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t* r, const void* smem_row) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -247,7 +256,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int KPW>
+template <int KPW, bool kHalf>
 __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const __grid_constant__ GlobalRowParams p) {
     constexpr int KP = kGrKeys / KPW;    // key slices of a chunk
     constexpr int RG = kGrWarps / KP;    // row tiles of 16 queries
@@ -346,7 +355,7 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks);
                     const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 16 * ks + 8);
-                    mma_bf16_16816(s[nt], qa[ks], b0, b1);
+                    mma_16816<kHalf>(s[nt], qa[ks], b0, b1);
                 }
             }
             // mask, scale, row maxima (each row's scores live in the 4 lanes of its quad)
@@ -394,8 +403,8 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
                     const float e2 = exp2f(sv[2] - bs_b), e3 = exp2f(sv[3] - bs_b);
                     l_a += e0 + e1;
                     l_b += e2 + e3;
-                    pa[kk][2 * h] = pack_bf16x2(e0, e1);
-                    pa[kk][2 * h + 1] = pack_bf16x2(e2, e3);
+                    pa[kk][2 * h] = pack16x2<kHalf>(e0, e1);
+                    pa[kk][2 * h + 1] = pack16x2<kHalf>(e2, e3);
                 }
             }
             // O += P V: for each 16-key step, two 8-column tiles of V per ldmatrix
@@ -407,8 +416,8 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
                     uint32_t vf[4];
                     ldmatrix_x4_trans(vf, Vs + (k0 + 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1)) * kGrStride +
                                               8 * (nd + (lane >> 4)));
-                    mma_bf16_16816(o[nd], a4, vf[0], vf[1]);
-                    mma_bf16_16816(o[nd + 1], a4, vf[2], vf[3]);
+                    mma_16816<kHalf>(o[nd], a4, vf[0], vf[1]);
+                    mma_16816<kHalf>(o[nd + 1], a4, vf[2], vf[3]);
                 }
             }
         }
@@ -500,6 +509,7 @@ __global__ void __launch_bounds__(kGrWarps * 32, 3) global_rows_mma_kernel(const
 // programmatic dependent: the split kernel lets it launch once every split
 // CTA is on its last chunk, so only griddepcontrol.wait separates the two.  All
 // its loads are issued before any value is used (one round trip to L2).
+template <bool kHalf>
 __global__ void __launch_bounds__(64) global_rows_merge_kernel(const __grid_constant__ GlobalRowParams p) {
     __shared__ float wsh[kMaxSplits];
     __shared__ float red[2];
@@ -544,7 +554,10 @@ __global__ void __launch_bounds__(64) global_rows_merge_kernel(const __grid_cons
         if (c + 1 < nsplit) acc1 = fmaf(wsh[c + 1], v[c + 1], acc1);
     }
     const float y = L > 0.f ? (acc0 + acc1) / L : 0.f;
-    reinterpret_cast<__nv_bfloat16*>(p.out)[(static_cast<size_t>(bh) * p.T + g) * 64 + tid] = __float2bfloat16_rn(y);
+    if constexpr (kHalf)
+        reinterpret_cast<__half*>(p.out)[(static_cast<size_t>(bh) * p.T + g) * 64 + tid] = __float2half_rn(y);
+    else
+        reinterpret_cast<__nv_bfloat16*>(p.out)[(static_cast<size_t>(bh) * p.T + g) * 64 + tid] = __float2bfloat16_rn(y);
 }
 
 }  // namespace lf

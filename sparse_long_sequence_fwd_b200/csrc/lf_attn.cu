@@ -79,7 +79,7 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
     Layout L{};
     L.W = (T + 31) / 32;
     L.gstride = std::max(1, std::min(n_global, T));
-    if (dtype == LF_BF16) {
+    if (dtype != LF_F32) {
         // tensor-core global rows: 128-key chunks, cpc per CTA, about three CTAs
         // per SM of a 148-SM B200 (each holds a two-stage ring of 72 KB)
         const int nblk = (T + kGrKeys - 1) / kGrKeys;
@@ -115,7 +115,7 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
     L.off_kg = o;
     L.off_vg = o;
     L.off_qg = o;
-    if (dtype == LF_BF16 && n_global > 0) {
+    if (dtype != LF_F32 && n_global > 0) {
         const size_t kgb = sizeof(__nv_bfloat16) * size_t(B) * H * L.ngp * 64;
         L.off_vg = align256(o + kgb);
         L.off_qg = align256(L.off_vg + kgb);
@@ -124,7 +124,7 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
     L.off_bcnt = o;
     L.off_bpart = o;
     L.band_tiles = 0;
-    if (dtype == LF_BF16) {
+    if (dtype != LF_F32) {
         // every head has at most ceil(T / 128) + kMaxDilTma - 1 tiles (one per residue class more)
         L.band_tiles = (long long)B * H * ((T + kBM - 1) / kBM + kMaxDilTma - 1);
         L.off_bpart = align256(o + sizeof(int32_t) * size_t(L.band_tiles) * 8);
@@ -145,26 +145,23 @@ bool is_capturing(cudaStream_t s) {
 lf_status set_kernel_attributes() {
     const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + 2 * kMaxGlobal) * 4;
     const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
-    if (cudaFuncSetAttribute(band_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(band_tc_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
-        cudaFuncSetAttribute(band_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(band_tc_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
-        cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) != cudaSuccess ||
+    for (auto kern : {band_tc_kernel<false, false>, band_tc_kernel<true, false>, band_tc_kernel<false, true>,
+                      band_tc_kernel<true, true>})
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+            return LF_ERR_CUDA;
+    for (auto kern : {global_rows_mma_kernel<32, false>, global_rows_mma_kernel<64, false>,
+                      global_rows_mma_kernel<128, false>, global_rows_mma_kernel<32, true>,
+                      global_rows_mma_kernel<64, true>, global_rows_mma_kernel<128, true>})
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) != cudaSuccess)
+            return LF_ERR_CUDA;
+    if (cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) != cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
             cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
             cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(global_rows_mma_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(global_rows_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(global_rows_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) !=
             cudaSuccess)
         return LF_ERR_CUDA;
     return LF_OK;
@@ -228,15 +225,16 @@ lf_status get_encoder() {
     return LF_OK;
 }
 
-// 3-D bf16 map over [d=64, rows, B*H] with a 128-byte swizzle; box = 64 x
-// (rows_per_box * stride) x 1, element stride `stride` along the rows.
+// 3-D map of 16-bit elements (bf16, or f16 when half) over [d=64, rows, B*H]
+// with a 128-byte swizzle; box = 64 x (rows_per_box * stride) x 1, element
+// stride `stride` along the rows.
 lf_status encode_rows_map(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t bh, uint32_t rows_per_box,
-                          uint32_t stride) {
+                          uint32_t stride, bool half) {
     cuuint64_t gdim[3] = {64, rows, bh};
     cuuint64_t gstr[2] = {64 * 2, rows * 64 * 2};
     cuuint32_t box[3] = {64, rows_per_box * stride, 1};
     cuuint32_t estr[3] = {1, stride, 1};
-    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstr, box, estr,
+    CUresult r = g_encode(tm, half ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstr, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? LF_OK : LF_ERR_CUDA;
@@ -249,7 +247,7 @@ lf_status check_args(const void* q, const void* k, const void* v, void* out, int
     if (n_global > 0 && !gidx) return LF_ERR_INVALID_ARG;
     if (n_global == 0 && gidx) return LF_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return LF_ERR_INVALID_ARG;
-    if (dtype != LF_F32 && dtype != LF_BF16) return LF_ERR_INVALID_ARG;
+    if (dtype != LF_F32 && dtype != LF_BF16 && dtype != LF_F16) return LF_ERR_INVALID_ARG;
     if (dil)
         for (int h = 0; h < H; ++h)
             if (dil[h] < 1) return LF_ERR_INVALID_ARG;
@@ -262,7 +260,7 @@ lf_status check_args(const void* q, const void* k, const void* v, void* out, int
     if (uint64_t(B) * H > 0x7fffffffull || uint64_t(B) * H * T > (uint64_t(1) << 31) * 64) return LF_ERR_UNSUPPORTED;
     if (dtype == LF_F32 && d > 128) return LF_ERR_UNSUPPORTED;
     if (n_global > 0 && uint64_t(B) * H > 65535u) return LF_ERR_UNSUPPORTED;  // global-row grid.y
-    if (dtype == LF_BF16) {
+    if (dtype != LF_F32) {  // the tensor-core path, bf16 or f16
         if (d != 64 || H > kMaxHeads) return LF_ERR_UNSUPPORTED;
         int kinds[kMaxDilKinds];
         int nk = 0;
@@ -375,6 +373,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
     ws.vg = reinterpret_cast<__nv_bfloat16*>(base + L.off_vg);
     ws.qg = reinterpret_cast<__nv_bfloat16*>(base + L.off_qg);
     const int r_eff = std::min(r, T);  // a window wider than the sequence changes nothing
+    const bool half = dtype == LF_F16;
     const float sl2 = static_cast<float>(double(scale) * kLog2e);
     int launches = 0;
 
@@ -392,7 +391,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
     pp.gstride = L.gstride;
     pp.ngp = L.ngp;
     pp.W = L.W;
-    pp.pack = (dtype == LF_BF16 && n_global > 0) ? 1 : 0;
+    pp.pack = (dtype != LF_F32 && n_global > 0) ? 1 : 0;
     pp.band_cnt = reinterpret_cast<int32_t*>(base + L.off_bcnt);
     pp.n_band_cnt = static_cast<int>(L.band_tiles * 8);
     const size_t prep_smem = size_t(L.W + 2 * kPrepThreads + 2 * L.gstride) * 4;
@@ -404,7 +403,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
     // here and joined after the band kernel, which is launched first and so
     // takes the SMs first.
     const bool global_stage = n_global > 0 && (stages & 4u);
-    const bool fork = global_stage && (stages & 2u) && dtype == LF_BF16 && ds->aux != nullptr;
+    const bool fork = global_stage && (stages & 2u) && dtype != LF_F32 && ds->aux != nullptr;
     if (fork && cudaEventRecord(ds->ev_fork, stream) != cudaSuccess) return LF_ERR_CUDA;
 
     if (!(stages & 2u)) {
@@ -431,7 +430,7 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         else band_f32_kernel<128><<<grid, kBandF32Warps * 32, 0, stream>>>(bp);
         ++launches;
     } else {
-        // K1: bf16 band rows on the tensor cores
+        // K1: bf16 or f16 band rows on the tensor cores
         st = get_encoder();
         if (st != LF_OK) return st;
         static thread_local BandTcParams bp;  // large (tensor maps); filled per call
@@ -441,9 +440,9 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         for (int kd = 0; kd < nk; ++kd) {
             const int dl = bp.dk_dil[kd];
             const uint32_t R = static_cast<uint32_t>(bp.dk_rows[kd]);
-            if ((st = encode_rows_map(&bp.tm_q[kd], q, T, uint64_t(B) * H, R, dl)) != LF_OK ||
-                (st = encode_rows_map(&bp.tm_k[kd], k, T, uint64_t(B) * H, R, dl)) != LF_OK ||
-                (st = encode_rows_map(&bp.tm_v[kd], v, T, uint64_t(B) * H, R, dl)) != LF_OK)
+            if ((st = encode_rows_map(&bp.tm_q[kd], q, T, uint64_t(B) * H, R, dl, half)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_k[kd], k, T, uint64_t(B) * H, R, dl, half)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_v[kd], v, T, uint64_t(B) * H, R, dl, half)) != LF_OK)
                 return st;
         }
         for (int a = nk; a < kMaxDilKinds; ++a) {  // unused slots: valid maps, never read
@@ -452,8 +451,8 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
             bp.tm_v[a] = bp.tm_v[0];
         }
         if (n_global > 0) {
-            if ((st = encode_rows_map(&bp.tm_kg, ws.kg, L.ngp, uint64_t(B) * H, kBN, 1)) != LF_OK ||
-                (st = encode_rows_map(&bp.tm_vg, ws.vg, L.ngp, uint64_t(B) * H, kBN, 1)) != LF_OK)
+            if ((st = encode_rows_map(&bp.tm_kg, ws.kg, L.ngp, uint64_t(B) * H, kBN, 1, half)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_vg, ws.vg, L.ngp, uint64_t(B) * H, kBN, 1, half)) != LF_OK)
                 return st;
         } else {
             bp.tm_kg = bp.tm_k[0];
@@ -491,8 +490,10 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         // more than 32 global tokens: the instantiation whose global-key dedup searches
-        if (cudaLaunchKernelEx(&cfg, n_global > 32 ? band_tc_kernel<true> : band_tc_kernel<false>, bp) != cudaSuccess)
-            return LF_ERR_CUDA;
+        void (*kern)(BandTcParams) =
+            n_global > 32 ? (half ? band_tc_kernel<true, true> : band_tc_kernel<true, false>)
+                          : (half ? band_tc_kernel<false, true> : band_tc_kernel<false, false>);
+        if (cudaLaunchKernelEx(&cfg, kern, bp) != cudaSuccess) return LF_ERR_CUDA;
         ++launches;
     }
 
@@ -516,13 +517,15 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         gp.sl2 = sl2;
         gp.cpc = L.cpc;
         gp.ngp = L.ngp;
-        if (dtype == LF_BF16) {
+        if (dtype != LF_F32) {
             // key splits x (b, h) x groups of kpw / 2 global rows, then the merge of the splits
             const int kpw = L.gr_kpw, rows = kpw / 2;
             const dim3 grid(L.nchunk, B * H, (L.gstride + rows - 1) / rows);
-            if (kpw == 32) global_rows_mma_kernel<32><<<grid, kGrWarps * 32, kGrSmem, gs>>>(gp);
-            else if (kpw == 64) global_rows_mma_kernel<64><<<grid, kGrWarps * 32, kGrSmem, gs>>>(gp);
-            else global_rows_mma_kernel<128><<<grid, kGrWarps * 32, kGrSmem, gs>>>(gp);
+            void (*grk)(GlobalRowParams) =
+                kpw == 32 ? (half ? global_rows_mma_kernel<32, true> : global_rows_mma_kernel<32, false>)
+                : kpw == 64 ? (half ? global_rows_mma_kernel<64, true> : global_rows_mma_kernel<64, false>)
+                            : (half ? global_rows_mma_kernel<128, true> : global_rows_mma_kernel<128, false>);
+            grk<<<grid, kGrWarps * 32, kGrSmem, gs>>>(gp);
             // the merge is the split kernel's programmatic dependent: it launches while the
             // splits finish and waits for them (griddepcontrol.wait) before reading
             cudaLaunchConfig_t mc = {};
@@ -534,7 +537,9 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
             mattr[0].val.programmaticStreamSerializationAllowed = 1;
             mc.attrs = mattr;
             mc.numAttrs = 1;
-            if (cudaLaunchKernelEx(&mc, global_rows_merge_kernel, gp) != cudaSuccess) return LF_ERR_CUDA;
+            if (cudaLaunchKernelEx(&mc, half ? global_rows_merge_kernel<true> : global_rows_merge_kernel<false>, gp) !=
+                cudaSuccess)
+                return LF_ERR_CUDA;
             launches += 2;
         } else {
             const dim3 grid(L.nchunk, B * H);
@@ -634,7 +639,7 @@ lf_status lf_attn_fwd_host(const void* q, const void* k, const void* v, void* ou
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceState* ds = nullptr;
     if ((st = device_state(&ds)) != LF_OK) return st;
-    const size_t es = dtype == LF_BF16 ? 2 : 4;
+    const size_t es = dtype == LF_F32 ? 4 : 2;
     const size_t nb = size_t(B) * H * T * d * es;
     const size_t o_q = 0, o_k = align256(nb), o_v = 2 * align256(nb), o_o = 3 * align256(nb);
     const size_t o_g = 4 * align256(nb);

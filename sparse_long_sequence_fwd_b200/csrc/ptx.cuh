@@ -188,13 +188,17 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
                      "l"(bdesc), "r"(idesc));
 }
 
-// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
+// Instruction descriptor, kind::f16: bf16 x bf16 (or, idesc_f16, f16 x f16) -> fp32, dense.
 //   [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
 //   15 A major (0 = K), 16 B major (1 = MN), [17,23) N >> 3, [24,29) M >> 4.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
            (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same with A and B in f16 (format 0).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn) {
+    return idesc_bf16(M, N, a_mn, b_mn) & ~((7u << 7) | (7u << 10));
 }
 
 // Shared-memory matrix descriptors for 128-byte-swizzled tiles whose rows
@@ -385,6 +389,18 @@ __device__ __forceinline__ float ex2_approx(float x) {  // hardware 2^x (MUFU)
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&t);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 t = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&t);
+}
+// Two values rounded to the 16-bit input type (kHalf: f16, else bf16), packed.
+template <bool kHalf>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi) {
+    if constexpr (kHalf)
+        return pack_f16x2(lo, hi);
+    else
+        return pack_bf16x2(lo, hi);
 }
 
 }  // namespace lf

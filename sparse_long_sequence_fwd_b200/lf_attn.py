@@ -15,7 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "liblfattn.so")
 
-LF_F32, LF_BF16 = 0, 1
+LF_F32, LF_BF16, LF_F16 = 0, 1, 2
 STATUS = {0: "LF_OK", 1: "LF_ERR_INVALID_ARG", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
           4: "LF_ERR_NO_MEMORY", 5: "LF_ERR_DEVICE_CHECK", 6: "LF_ERR_SCRATCH_TOO_SMALL"}
 EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
@@ -79,7 +79,9 @@ def _dtype_code(t: torch.Tensor) -> int:
         return LF_F32
     if t.dtype == torch.bfloat16:
         return LF_BF16
-    raise TypeError("q/k/v must be float32 or bfloat16, got %s" % t.dtype)
+    if t.dtype == torch.float16:
+        return LF_F16
+    raise TypeError("q/k/v must be float32, bfloat16 or float16, got %s" % t.dtype)
 
 
 def _dil_array(dil, H):

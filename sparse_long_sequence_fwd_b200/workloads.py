@@ -9,8 +9,9 @@ Recipe (the same for every workload):
   * ``g = torch.Generator().manual_seed(seed)``;
   * ``q``, ``k``, ``v`` drawn in that order with ``torch.randn(B, H, T, d,
     generator=g)`` (fp32, iid N(0, 1));
-  * bf16 workloads round them with ``.to(torch.bfloat16)`` (round to nearest
-    even); the oracle reads those rounded values widened to fp64;
+  * bf16 workloads round them with ``.to(torch.bfloat16)`` and f16 workloads
+    with ``.to(torch.float16)`` (round to nearest even); the oracle reads those
+    rounded values widened to fp64;
   * random global positions (if any) are drawn from the same generator after
     v, with ``torch.randperm``;
   * the key padding mask is uint8 [B, T], nonzero = padded key.
@@ -34,7 +35,7 @@ import torch
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    dtype: str                      # "f32" or "bf16"
+    dtype: str                      # "f32", "bf16" or "f16"
     B: int
     H: int
     T: int
@@ -74,14 +75,18 @@ DILATED = Workload("dilated_T8192_r128", "bf16", 1, 12, 8192, 64, 128,
 LARGE = Workload("large_T16384_g32", "bf16", 1, 16, 16384, 64, 256, _dil(16, 1),
                  globals_per_b=None, n_random_globals=32, scale=0.125, seed=1005)
 
-ALL = [TINY, BASE, QA, DILATED, LARGE]
+# the base workload with f16 inputs (the pages train with fp16 mixed
+# precision: Longformer wiki, section 6.3)
+BASE_F16 = dataclasses.replace(BASE, name="base_T4096_w513_f16", dtype="f16")
+
+ALL = [TINY, BASE, QA, DILATED, LARGE, BASE_F16]
 BY_NAME = {w.name: w for w in ALL}
 
 
 def make_inputs(w: Workload, device: str = "cpu"):
     """Seeded inputs for a workload.
 
-    Returns a dict with ``q, k, v`` ([B, H, T, d], fp32 or bf16),
+    Returns a dict with ``q, k, v`` ([B, H, T, d], fp32, bf16 or f16),
     ``global_idx`` (int32 [B, n_global] or None), ``key_pad_mask``
     (uint8 [B, T] or None) and ``dil`` (int32 [H], host).
     """
@@ -92,6 +97,8 @@ def make_inputs(w: Workload, device: str = "cpu"):
     v = torch.randn(shape, generator=g)
     if w.dtype == "bf16":
         q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    elif w.dtype == "f16":
+        q, k, v = (t.to(torch.float16) for t in (q, k, v))
     elif w.dtype != "f32":
         raise ValueError(w.dtype)
 

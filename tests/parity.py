@@ -8,6 +8,10 @@ from sparse_long_sequence_fwd_b200 import lf_attn, workloads
 
 BF16_MAX_ABS = 2e-2
 BF16_REL_RMS = 5e-3
+# f16 rounds with unit 2^-11 where bf16 rounds with 2^-8 (inputs, P, output):
+# the bf16 bar scaled by 1/8, with some room
+F16_MAX_ABS = 4e-3
+F16_REL_RMS = 1e-3
 F32_MAX_ABS = 1e-5
 
 
@@ -40,6 +44,9 @@ def compare(w, got, ref):
     rel_rms = float(np.sqrt((diff ** 2).sum()) / denom) if denom > 0 else float(np.sqrt((diff ** 2).sum()))
     if w.dtype == "f32":
         assert max_abs <= F32_MAX_ABS, (max_abs, np.unravel_index(diff.argmax(), diff.shape))
+    elif w.dtype == "f16":
+        assert max_abs <= F16_MAX_ABS, (max_abs, np.unravel_index(diff.argmax(), diff.shape))
+        assert rel_rms <= F16_REL_RMS, rel_rms
     else:
         assert max_abs <= BF16_MAX_ABS, (max_abs, np.unravel_index(diff.argmax(), diff.shape))
         assert rel_rms <= BF16_REL_RMS, rel_rms

@@ -39,6 +39,8 @@ def test_strerror_and_workspace(lib):
         assert lf_attn.strerror(code)
     assert lib.lf_attn_workspace_bytes(1, 12, 4096, 64, 1, 1) > 0
     assert lib.lf_attn_workspace_bytes(0, 12, 4096, 64, 1, 1) == 0
+    # f16 uses the tensor-core path's workspace, the same as bf16
+    assert lib.lf_attn_workspace_bytes(2, 12, 4096, 64, 64, 2) == lib.lf_attn_workspace_bytes(2, 12, 4096, 64, 64, 1)
 
 
 FAKE = 1 << 20  # aligned non-null address, never dereferenced by the argument checks
@@ -63,6 +65,8 @@ def _call(lib, **kw):
     (dict(d=32), 2), (dict(d=128), 2),                                           # bf16 path: d == 64 only
     (dict(dil=(ctypes.c_int32 * 2)(1, 9)), 2),                                   # TMA element stride <= 8
     (dict(T=(1 << 20) + 1), 2), (dict(H=129), 2), (dict(dtype=0, d=129), 2),
+    (dict(dtype=2, d=128), 2), (dict(dtype=2, dil=(ctypes.c_int32 * 2)(1, 9)), 2),  # f16: same limits as bf16
+    (dict(dtype=3), 1),
 ])
 def test_argument_errors_return_status_without_launch(lib, kw, code):
     assert _call(lib, **kw) == code

@@ -12,6 +12,8 @@
 bf16 bar: max-abs <= 2e-2 and relative RMS <= 5e-3 over the whole tensor
 (over the compared rows for the sampled-row check).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -65,7 +67,7 @@ SMALL = [
 
 
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
-def test_small_cases_every_element(w):
+def test_small_cases_full_case(w):
     _full_case(w)
 
 
@@ -74,7 +76,7 @@ def test_base_workload_every_element():
 
 
 @pytest.mark.parametrize("w", [workloads.QA, workloads.DILATED, workloads.LARGE], ids=lambda w: w.name)
-def test_full_size_workloads_every_element(w):
+def test_full_size_workloads_full_case(w):
     """QA (two samples, 64 globals, padding), dilated (dilation 1 and 2) and
     large (T = 16384, 32 random globals): every element of the output against
     the full oracle, max-abs and relative RMS over the whole tensor."""
@@ -122,7 +124,7 @@ EDGES = [
 
 
 @pytest.mark.parametrize("w", EDGES, ids=lambda w: w.name)
-def test_edge_cases_every_element(w):
+def test_edge_cases_full_case(w):
     _full_case(w)
 
 
@@ -246,12 +248,13 @@ def test_output_guard_regions_untouched():
     parity.compare(w, out, parity.oracle_full(w, inp))
 
 
-def test_host_entry_point_matches_device_entry_point():
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_host_entry_point_matches_device_entry_point(dtype):
     """The host entry point runs the call as slices of (sample, heads), one
     launch each, so the band kernel splits its work differently from one
     whole launch and split tiles merge in another order: both entry points
     are compared with the oracle, and with each other at the same bar."""
-    w = workloads.custom("host_api", "bf16", 2, 2, 700, 64, 60, globals_per_b=[[0, 5], [9, 9]],
+    w = workloads.custom("host_api", dtype, 2, 2, 700, 64, 60, globals_per_b=[[0, 5], [9, 9]],
                          pad_from=[None, 600], seed=42)
     inp = workloads.make_inputs(w)
     dev = parity.run_gpu(w, inp)
@@ -293,3 +296,28 @@ def test_argument_errors_on_gpu_do_not_launch():
     assert e.value.status == 2
     st, flags = lf_attn.device_status()
     assert st == 0 and flags == 0
+
+
+# f16 inputs (the pages train with fp16 mixed precision: Longformer wiki,
+# section 6.3): the same tensor-core kernels instantiated for f16 operands.
+F16_CASES = [
+    workloads.custom("f16_multi_tile", "f16", 2, 3, 1000, 64, 100, dil=[1, 2, 3],
+                     globals_per_b=[[0, 999, 500, 500], [7, 3, 3, 640]], pad_from=[None, 777], seed=51),
+    workloads.custom("f16_49_globals_dil", "f16", 2, 4, 1500, 64, 60, dil=[1, 2, 3, 4],
+                     globals_per_b=[list(range(5, 1500, 31)) + [5, 36], list(range(700, 1100, 9)) + [1096] * 6],
+                     pad_from=[1400, None], seed=52),
+    workloads.custom("f16_r256_scale_neg", "f16", 1, 2, 900, 64, 256, globals_per_b=[[3, 899]], scale=-0.3,
+                     seed=53),
+    workloads.custom("f16_no_globals_T129", "f16", 1, 2, 129, 64, 128, seed=54),
+]
+
+
+@pytest.mark.parametrize("w", F16_CASES, ids=lambda w: w.name)
+def test_f16_cases_full_case(w):
+    _full_case(w)
+
+
+@pytest.mark.parametrize("base", [workloads.BASE, workloads.QA], ids=lambda w: w.name)
+def test_f16_full_size_every_element(base):
+    w = dataclasses.replace(base, name=base.name + "_f16", dtype="f16")
+    _full_case(w)
