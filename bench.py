@@ -59,7 +59,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-others", action="store_true",
-                    help="skip the QA, dilated, large and f16 base workload entries")
+                    help="skip the QA, dilated, large, f16 base and d = 128 workload entries")
     return ap.parse_args()
 
 
@@ -395,7 +395,8 @@ def run_ours(args):
     # ---- the other workloads (each its own rotating inputs), rank 0 only
     others = {}
     if rank == 0 and world == 1 and not args.no_others:
-        for name in ("qa_B2_T4096_g64_pad", "dilated_T8192_r128", "large_T16384_g32", "base_T4096_w513_f16"):
+        for name in ("qa_B2_T4096_g64_pad", "dilated_T8192_r128", "large_T16384_g32", "base_T4096_w513_f16",
+                     "d128_H8_T4096_w513"):
             if name == w.name:
                 continue
             ow = workloads.BY_NAME[name]

@@ -70,9 +70,10 @@ typedef enum {
  *   key_pad_mask DEVICE uint8 [B, T], nonzero = padded key; NULL = none
  *   scale       softmax scale (usually 1/sqrt(d))
  *   dtype       LF_F32: CUDA-core fp32 path, d <= 128.
- *               LF_BF16: tensor-core path (tcgen05 + TMA), d == 64 only,
+ *               LF_BF16: tensor-core path (tcgen05 + TMA), d == 64 or 128,
  *               fp32 accumulation and softmax, every dil[h] <= 8, at most 4
- *               distinct dilation values, H <= 128.
+ *               distinct dilation values, H <= 128.  (d == 128 runs one band
+ *               CTA per SM, and its global rows on the CUDA cores.)
  *               LF_F16: the same tensor-core path with fp16 q, k, v and out
  *               (fp16 MMA operands, the probabilities rounded to fp16 for the
  *               P V product), with the same limits.  The pages train with

@@ -59,49 +59,62 @@ namespace lf {
 
 constexpr int kBM = 128;  // queries per tile
 constexpr int kBN = 64;   // keys per block
-constexpr int kHD = 64;
 constexpr int kQStages = 2;
 constexpr int kKVStages = 4;
 constexpr int kSBufs = 3;                // S / P buffers in TMEM
-constexpr int kQBytes = kBM * kHD * 2;   // 16 KB: 128 rows x 128 bytes
-constexpr int kKVBytes = kBN * kHD * 2;  // 8 KB
 constexpr int kBandThreads = 192;
-constexpr int kBandCtasPerSm = 2;
 constexpr int kSoftmaxWarps = 4;
 constexpr float kRescaleLog2 = 8.f;  // move the exponent base only past 2^8
 
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQStages * kQBytes;
-constexpr int kOffV = kOffK + kKVStages * kKVBytes;
-constexpr int kOffBar = kOffV + kKVStages * kKVBytes;
 // barrier slots
 constexpr int kBarQFull = 0, kBarQEmpty = kBarQFull + kQStages, kBarKFull = kBarQEmpty + kQStages,
               kBarKEmpty = kBarKFull + kKVStages, kBarVFull = kBarKEmpty + kKVStages,
               kBarVEmpty = kBarVFull + kKVStages, kBarSFull = kBarVEmpty + kKVStages, kBarPFull = kBarSFull + kSBufs,
               kBarBufFree = kBarPFull + kSBufs, kBarOFull = kBarBufFree + kSBufs, kBarDrain = kBarOFull + 2,
               kNumBars = kBarDrain + 1;
-// Piece descriptors (BandPiece), one per Q slot: written by the producer
-// before it arrives on the slot's Q-full barrier, read by the MMA and softmax
-// roles after waiting on it, so only the producer walks the work sequence.
-// A slot (Q tile and descriptor) is free again once the piece's last
-// product has been issued and its rows have been written.
-constexpr int kOffDesc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
 constexpr int kDescBytes = 128;
-constexpr int kOffMisc = kOffDesc + kQStages * kDescBytes;
 constexpr int kMiscBytes = 16;
-constexpr int kBandSmem = kOffMisc + kMiscBytes + 1024;  // + alignment slack
-static_assert(kBandCtasPerSm * (kBandSmem + 1024) <= 233472, "shared memory budget for two CTAs per SM");
-
-// TMEM columns (256 per CTA): three S buffers of 64 fp32 columns at 0, 64,
-// 128 (P, bf16 pairs, over the first 32 columns of its own buffer), O (fp32,
-// 64 wide) at 192.
-constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 192;
 
-// Partial state of one piece (128 rows): O as [16][128][4] fp32 (four
-// columns of every row per 16-byte group, so a warp's stores and loads are
-// contiguous), then m[128] and l[128].
-constexpr int kPartFloats = kBM * kHD + 2 * kBM;
+// What depends on the head dimension HD (64 or 128).  Rows of q, k and v are
+// staged as HD / 64 sub-tiles of 64 columns (128 bytes, one 128-byte swizzle
+// atom per row), each a separate TMA box and MMA operand.
+//   Shared memory: Q tiles (kQStages), then the K and V rings (kKVStages),
+//   the barriers, the piece descriptors (one per Q slot: written by the
+//   producer before it arrives on the slot's Q-full barrier, read by the MMA
+//   and softmax roles after waiting on it, so only the producer walks the
+//   work sequence; a slot is free again once the piece's last product has
+//   been issued and its rows have been written), then the TMEM slot and the
+//   abort flag.
+//   TMEM: three S buffers of 64 fp32 columns at 0, 64, 128 (P, 16-bit pairs,
+//   over the first 32 columns of its own buffer), O (fp32, HD wide) at 192:
+//   256 columns, two CTAs per SM, for HD = 64; 320 (a 512-column
+//   allocation), one CTA per SM, for HD = 128.
+//   Partial state of one piece (128 rows): O as [HD / 4][128][4] fp32 (four
+//   columns of every row per 16-byte group, so a warp's stores and loads are
+//   contiguous), then m[128] and l[128].
+template <int HD>
+struct BandCfg {
+    static_assert(HD == 64 || HD == 128, "head dimension");
+    static constexpr int kHD = HD;
+    static constexpr int kSub = HD / 64;            // 64-column sub-tiles per row
+    static constexpr int kQBytes = kBM * HD * 2;    // 16 KB per 64 columns: 128 rows x 128 bytes
+    static constexpr int kQSubBytes = kBM * 128;
+    static constexpr int kKVBytes = kBN * HD * 2;   // 8 KB per 64 columns
+    static constexpr int kKVSubBytes = kBN * 128;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQStages * kQBytes;
+    static constexpr int kOffV = kOffK + kKVStages * kKVBytes;
+    static constexpr int kOffBar = kOffV + kKVStages * kKVBytes;
+    static constexpr int kOffDesc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
+    static constexpr int kOffMisc = kOffDesc + kQStages * kDescBytes;
+    static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+    static constexpr int kCtasPerSm = HD == 64 ? 2 : 1;
+    static constexpr uint32_t kTmemCols = HD == 64 ? 256 : 512;
+    static constexpr int kPartFloats = kBM * HD + 2 * kBM;
+    static_assert(kCtasPerSm * (kSmem + 1024) <= 233472, "shared memory budget per SM");
+    static_assert(kColO + HD <= kTmemCols, "TMEM budget");
+};
 
 // One piece: blocks [blk_lo, blk_hi) of one tile's nbb band blocks and ngb
 // global blocks.
@@ -285,8 +298,10 @@ __device__ __forceinline__ float min32(const uint32_t* v) {
 // Only the global-key blocks read the prep kernel's output (packed keys), so
 // the wait for prep comes just before the first of them: the band blocks of
 // the first tile overlap prep.
+template <int HD>
 __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                               volatile int* abort_flag) {
+    using C = BandCfg<HD>;
     const int s = blockIdx.x;
     const int x0 = range_start(p, s);
     const int x1 = range_start(p, s + 1);
@@ -306,20 +321,25 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
         uint64_t* empty = &bars[(is_v ? kBarVEmpty : kBarKEmpty) + st];
         uint64_t* full = &bars[(is_v ? kBarVFull : kBarKFull) + st];
         if (!mbar_wait(empty, ph ^ 1u, abort_flag, p.wait_ns)) return false;
-        uint8_t* dst = smem + (is_v ? kOffV : kOffK) + st * kKVBytes;
+        uint8_t* dst = smem + (is_v ? C::kOffV : C::kOffK) + st * C::kKVBytes;
         if (blk < d.nbb) {
-            mbar_arrive_expect_tx(full, kKVBytes);
+            mbar_arrive_expect_tx(full, C::kKVBytes);
             const int j0 = d.kbase + kBN * (d.kb_lo + blk);
             const CUtensorMap* tm = is_v ? &p.tm_v[d.dk] : &p.tm_k[d.dk];
-            for (int u = 0; u < kBN; u += d.R)
-                tma_load_3d(dst + u * 128, tm, full, 0, d.c + d.dil * (j0 + u), d.bh);
+#pragma unroll
+            for (int sub = 0; sub < C::kSub; ++sub)
+                for (int u = 0; u < kBN; u += d.R)
+                    tma_load_3d(dst + sub * C::kKVSubBytes + u * 128, tm, full, 64 * sub, d.c + d.dil * (j0 + u), d.bh);
         } else {
             if (!prep_done) {  // packed global keys from here on
                 grid_dep_wait();
                 prep_done = true;
             }
-            mbar_arrive_expect_tx(full, kKVBytes);
-            tma_load_3d(dst, is_v ? &p.tm_vg : &p.tm_kg, full, 0, (blk - d.nbb) * kBN, d.bh);
+            mbar_arrive_expect_tx(full, C::kKVBytes);
+#pragma unroll
+            for (int sub = 0; sub < C::kSub; ++sub)
+                tma_load_3d(dst + sub * C::kKVSubBytes, is_v ? &p.tm_vg : &p.tm_kg, full, 64 * sub, (blk - d.nbb) * kBN,
+                            d.bh);
         }
         return true;
     };
@@ -368,16 +388,19 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
                 d.s1 = s1;
                 d.last = (!in_front && pend == x_main_end) ? 1 : 0;
                 d.tstart = cw->start;
-                *reinterpret_cast<BandPiece*>(smem + kOffDesc + qs * kDescBytes) = d;  // released by the arrive
-                mbar_arrive_expect_tx(&bars[kBarQFull + qs], kQBytes);
-                uint8_t* dQ = smem + kOffQ + qs * kQBytes;
-                for (int u = 0; u < kBM; u += d.R)
-                    tma_load_3d(dQ + u * 128, &p.tm_q[d.dk], &bars[kBarQFull + qs], 0, d.c + d.dil * (d.q0 + u), d.bh);
+                *reinterpret_cast<BandPiece*>(smem + C::kOffDesc + qs * kDescBytes) = d;  // released by the arrive
+                mbar_arrive_expect_tx(&bars[kBarQFull + qs], C::kQBytes);
+                uint8_t* dQ = smem + C::kOffQ + qs * C::kQBytes;
+#pragma unroll
+                for (int sub = 0; sub < C::kSub; ++sub)
+                    for (int u = 0; u < kBM; u += d.R)
+                        tma_load_3d(dQ + sub * C::kQSubBytes + u * 128, &p.tm_q[d.dk], &bars[kBarQFull + qs], 64 * sub,
+                                    d.c + d.dil * (d.q0 + u), d.bh);
                 ++qt;
             }
             cur_slot = (qt - 1) & 1u;
             cur_blk = blk;
-            const BandPiece& d = *reinterpret_cast<const BandPiece*>(smem + kOffDesc + cur_slot * kDescBytes);
+            const BandPiece& d = *reinterpret_cast<const BandPiece*>(smem + C::kOffDesc + cur_slot * kDescBytes);
             if (!issue_kv(d, blk, false, gk)) break;
             ++gk;
             ++x;
@@ -394,7 +417,7 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
             }
         }
         if (have_prev) {
-            const BandPiece& d = *reinterpret_cast<const BandPiece*>(smem + kOffDesc + prev_slot * kDescBytes);
+            const BandPiece& d = *reinterpret_cast<const BandPiece*>(smem + C::kOffDesc + prev_slot * kDescBytes);
             if (!issue_kv(d, prev_blk, true, gv)) break;
             ++gv;
         }
@@ -420,16 +443,21 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
 // O-complete barrier of its parity (two barriers, so a softmax thread that
 // only sometimes waits for a product can still tell the phases apart).
 // kHalf: q, k, v (and so P) are f16 instead of bf16.
-template <bool kHalf>
+// With HD = 128, S sums the products of the two 64-column sub-tiles of Q and
+// K, and O's two 64-column halves each take the product with their own
+// sub-tile of V.
+template <bool kHalf, int HD>
 __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                          volatile int* abort_flag, uint32_t tmem_base) {
-    const uint32_t idesc_pv = kHalf ? idesc_f16(kBM, kHD, 0, 1) : idesc_bf16(kBM, kHD, 0, 1);
+    using C = BandCfg<HD>;
+    const uint32_t idesc_pv = kHalf ? idesc_f16(kBM, 64, 0, 1) : idesc_bf16(kBM, 64, 0, 1);
     uint64_t dQ[kQStages];
 #pragma unroll
-    for (int st = 0; st < kQStages; ++st) dQ[st] = sdesc_k_sw128(smem_u32(smem + kOffQ + st * kQBytes));
-    const uint64_t dK0 = sdesc_k_sw128(smem_u32(smem + kOffK));
-    const uint64_t dV0 = sdesc_mn_sw128(smem_u32(smem + kOffV));
-    constexpr uint64_t kKVDescStep = kKVBytes >> 4;  // start-address units per ring stage
+    for (int st = 0; st < kQStages; ++st) dQ[st] = sdesc_k_sw128(smem_u32(smem + C::kOffQ + st * C::kQBytes));
+    const uint64_t dK0 = sdesc_k_sw128(smem_u32(smem + C::kOffK));
+    const uint64_t dV0 = sdesc_mn_sw128(smem_u32(smem + C::kOffV));
+    constexpr uint64_t kKVDescStep = C::kKVBytes >> 4;  // start-address units per ring stage
+    constexpr uint64_t kQSubStep = C::kQSubBytes >> 4, kKVSubStep = C::kKVSubBytes >> 4;
     const uint32_t tO = tmem_base + kColO;
 
     // O += P(g) V(g) over nk keys; the first block of a piece overwrites O
@@ -439,13 +467,17 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
             !mbar_wait(&bars[kBarVFull + st], (g / kKVStages) & 1u, abort_flag, p.wait_ns))
             return false;
         tc_fence_after();
-        const uint64_t dv = dV0 + kKVDescStep * st;
         const uint32_t tP = tmem_base + 64u * b;
-        if (first)
-            tc_mma_ts<false>(tO, tP, dv, idesc_pv);
-        else
-            tc_mma_ts<true>(tO, tP, dv, idesc_pv);
-        for (int k = 1; k < nk / 16; ++k) tc_mma_ts<true>(tO, tP + 8u * k, dv + 128u * k, idesc_pv);
+#pragma unroll
+        for (int sub = 0; sub < C::kSub; ++sub) {
+            const uint64_t dv = dV0 + kKVDescStep * st + kKVSubStep * sub;
+            const uint32_t to = tO + 64u * sub;
+            if (first)
+                tc_mma_ts<false>(to, tP, dv, idesc_pv);
+            else
+                tc_mma_ts<true>(to, tP, dv, idesc_pv);
+            for (int k = 1; k < nk / 16; ++k) tc_mma_ts<true>(to, tP + 8u * k, dv + 128u * k, idesc_pv);
+        }
         tc_commit(&bars[kBarBufFree + b]);
         tc_commit(&bars[kBarOFull + (g & 1u)]);
         tc_commit(&bars[kBarVEmpty + st]);
@@ -459,7 +491,7 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
         const uint32_t qs = qt & 1u;
         if (!mbar_wait(&bars[kBarQFull + qs], (qt >> 1) & 1u, abort_flag, p.wait_ns)) break;
         ++qt;
-        const BandPiece* d = reinterpret_cast<const BandPiece*>(smem + kOffDesc + qs * kDescBytes);
+        const BandPiece* d = reinterpret_cast<const BandPiece*>(smem + C::kOffDesc + qs * kDescBytes);
         const int blk_lo = d->blk_lo, blk_hi = d->blk_hi, nbb = d->nbb, bsm = d->b;
         int ngk = -1;  // global keys of this sample (prep's output), read at the first global block
         done = d->last != 0;
@@ -484,6 +516,14 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
             tc_mma<true>(tS, dq + 2, dk + 2, ids);
             tc_mma<true>(tS, dq + 4, dk + 4, ids);
             tc_mma<true>(tS, dq + 6, dk + 6, ids);
+#pragma unroll
+            for (int sub = 1; sub < C::kSub; ++sub) {  // the next 64 columns of q and k
+                const uint64_t dqs = dq + kQSubStep * sub, dks = dk + kKVSubStep * sub;
+                tc_mma<true>(tS, dqs + 0, dks + 0, ids);
+                tc_mma<true>(tS, dqs + 2, dks + 2, ids);
+                tc_mma<true>(tS, dqs + 4, dks + 4, ids);
+                tc_mma<true>(tS, dqs + 6, dks + 6, ids);
+            }
             tc_commit(&bars[kBarSFull + b]);
             tc_commit(&bars[kBarKEmpty + st]);
             if (blk == blk_hi - 1) tc_commit(&bars[kBarQEmpty + qs]);
@@ -507,11 +547,12 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
 // state) of a piece is written when the next piece starts, or at the end,
 // once the piece's last product has finished.
 
-// Multiplies this thread's row of O (64 fp32 columns) by alpha, in TMEM,
+// Multiplies this thread's row of O (HD fp32 columns) by alpha, in TMEM,
 // 16 columns at a time (few registers: it runs inside the block loop).
+template <int HD>
 __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 #pragma unroll 1
-    for (int part = 0; part < 4; ++part) {
+    for (int part = 0; part < HD / 16; ++part) {
         uint32_t o[16];
         tmem_ld16(tO + 16u * part, o);
         tmem_ld_wait16(o);
@@ -566,18 +607,20 @@ __device__ __forceinline__ void store_half_rows(__nv_bfloat16* row_ptr, bool wri
 
 // Partial slot of CTA s's piece of a tile that starts at tstart: 2s for the
 // piece at the start of s's range, 2s + 1 for the one at its end.
+template <int HD>
 __device__ __forceinline__ float* part_slot(const BandTcParams& p, int s, int tstart) {
     const int k = 2 * s + (tstart > range_start(p, s) ? 1 : 0);
-    return p.part + static_cast<size_t>(k) * kPartFloats;
+    return p.part + static_cast<size_t>(k) * BandCfg<HD>::kPartFloats;
 }
 
 // Output of a finished piece (warp-wide: every lane calls it): its
 // descriptor d stays in shared memory until this is done; m and l are this
 // thread's row's exponent base and sum.  The row is handled 32 output
 // dimensions at a time (registers: this runs with the next piece's state live).
-template <bool kHalf>
+template <bool kHalf, int HD>
 __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiece* d, float m, float l, uint32_t tO,
                                           int wq, int ticket, volatile int* abort_flag) {
+    constexpr int kHD = HD, kHalves = HD / 32;  // 32-column groups of a row
     const int lane = threadIdx.x & 31;
     const int x = wq * 32 + lane;
     const int self = static_cast<int>(blockIdx.x);
@@ -597,7 +640,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
     if (d->blk_lo == 0 && d->blk_hi == d->nbb + d->ngb) {  // the whole tile
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-        for (int hd = 0; hd < 2; ++hd) {
+        for (int hd = 0; hd < kHalves; ++hd) {
             float o[32];
             load_o(hd, o);
             store_half_rows<kHalf>(dst, write, hd, o, inv);
@@ -609,10 +652,10 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
     int* cnt = p.cnt + (static_cast<size_t>(d->tile) * 4 + wq) * 2;  // [0] arrivals, [1] lanes done writing
     const int npieces = s1 - s0 + 1;
     if (ticket < npieces - 1) {  // not the last to arrive: leave the partial state for the last
-        float* slot = part_slot(p, self, tstart);
+        float* slot = part_slot<HD>(p, self, tstart);
         float4* o4 = reinterpret_cast<float4*>(slot);
 #pragma unroll 1
-        for (int hd = 0; hd < 2; ++hd) {
+        for (int hd = 0; hd < kHalves; ++hd) {
             float o[32];
             load_o(hd, o);
 #pragma unroll
@@ -643,7 +686,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
     // summed in CTA order whichever piece merges (the same operations either way)
     if (npieces == 2 && ok) {  // the common case: one other piece
         const int so = self == s0 ? s1 : s0;
-        const float* slot = part_slot(p, so, tstart);
+        const float* slot = part_slot<HD>(p, so, tstart);
         const float4* o4 = reinterpret_cast<const float4*>(slot);
         const float mo = __ldcg(slot + kBM * kHD + x);
         const float lo = __ldcg(slot + kBM * kHD + kBM + x);
@@ -656,7 +699,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
         const float L = fmaf(w2, self_first ? lo : l, w1 * (self_first ? l : lo));
         const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll 1
-        for (int hd = 0; hd < 2; ++hd) {
+        for (int hd = 0; hd < kHalves; ++hd) {
             float4 v[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) v[u] = __ldcg(o4 + (8 * hd + u) * kBM + x);
@@ -676,21 +719,21 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
     } else {
         float M = m;
         for (int s = s0; s <= s1; ++s)
-            if (s != self && ok) M = fmaxf(M, __ldcg(part_slot(p, s, tstart) + kBM * kHD + x));
+            if (s != self && ok) M = fmaxf(M, __ldcg(part_slot<HD>(p, s, tstart) + kBM * kHD + x));
         const float Mu = M == -INFINITY ? 0.f : M;
         float L = 0.f;
         for (int s = s0; s <= s1; ++s) {
             if (s == self) {
                 L = fmaf(m == -INFINITY ? 0.f : ex2_approx(m - Mu), l, L);
             } else if (ok) {
-                const float* slot = part_slot(p, s, tstart);
+                const float* slot = part_slot<HD>(p, s, tstart);
                 const float ms = __ldcg(slot + kBM * kHD + x);
                 L = fmaf(ms == -INFINITY ? 0.f : ex2_approx(ms - Mu), __ldcg(slot + kBM * kHD + kBM + x), L);
             }
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll 1
-        for (int hd = 0; hd < 2; ++hd) {
+        for (int hd = 0; hd < kHalves; ++hd) {
             float acc[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) acc[c] = 0.f;
@@ -704,7 +747,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
                     continue;
                 }
                 if (!ok) continue;
-                const float* slot = part_slot(p, s, tstart);
+                const float* slot = part_slot<HD>(p, s, tstart);
                 const float ms = __ldcg(slot + kBM * kHD + x);
                 const float wv = ms == -INFINITY ? 0.f : ex2_approx(ms - Mu);
                 const float4* o4 = reinterpret_cast<const float4*>(slot);
@@ -729,7 +772,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
 
 // kSearch: the sample may have more than 32 global keys; the global-key block's
 // dedup then finds the keys in a row's window by binary search (below).
-template <bool kSearch, bool kHalf>
+template <bool kSearch, bool kHalf, int HD>
 __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                              volatile int* abort_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -779,8 +822,8 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
     int ticket = 0;       // merge ticket of the current piece (split pieces), taken at its last block
     int ticket_prev = 0;  // the previous piece's, kept until its rows are written
     auto finish_prev = [&]() {
-        const BandPiece* dq = reinterpret_cast<const BandPiece*>(smem + kOffDesc + prev_slot * kDescBytes);
-        flush_rows<kHalf>(p, dq, m_prev, l_prev, tO, wq, __shfl_sync(0xffffffffu, ticket_prev, 0), abort_flag);
+        const BandPiece* dq = reinterpret_cast<const BandPiece*>(smem + BandCfg<HD>::kOffDesc + prev_slot * kDescBytes);
+        flush_rows<kHalf, HD>(p, dq, m_prev, l_prev, tO, wq, __shfl_sync(0xffffffffu, ticket_prev, 0), abort_flag);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarQEmpty + prev_slot]);
         prev_slot = -1;
@@ -794,7 +837,7 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
             if (!wait_warp(&bars[kBarQFull + qs], (qt >> 1) & 1u)) return;
             ++qt;
         }
-        const BandPiece* dp = reinterpret_cast<const BandPiece*>(smem + kOffDesc + qs * kDescBytes);
+        const BandPiece* dp = reinterpret_cast<const BandPiece*>(smem + BandCfg<HD>::kOffDesc + qs * kDescBytes);
         if (have) done = dp->last != 0;
         const int blk_lo = have ? dp->blk_lo : 0, blk_hi = have ? dp->blk_hi : 1, nbb = dp->nbb;
         const int i = dp->c + dp->dil * (dp->q0 + x);  // this row's position in the sequence
@@ -995,7 +1038,7 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
             // ---- O is rescaled only once the previous product is done
             if (__any_sync(0xffffffffu, o_move)) {
                 if (!wait_product(g - 1)) return;
-                rescale_o(tO, alpha);
+                rescale_o<HD>(tO, alpha);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -1014,13 +1057,16 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
 
 // Instantiations from one source: kSearch = true for calls with more than 32
 // global tokens (see softmax_role), false otherwise, so each keeps its own
-// code for the block loop; kHalf = true for f16 inputs, false for bf16.
-template <bool kSearch, bool kHalf>
-__global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(const __grid_constant__ BandTcParams p) {
+// code for the block loop; kHalf = true for f16 inputs, false for bf16; HD =
+// the head dimension (64: two CTAs per SM; 128: one).
+template <bool kSearch, bool kHalf, int HD>
+__global__ void __launch_bounds__(kBandThreads, BandCfg<HD>::kCtasPerSm)
+    band_tc_kernel(const __grid_constant__ BandTcParams p) {
+    using C = BandCfg<HD>;
     extern __shared__ uint8_t band_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(band_smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     uint32_t* tmem_slot = misc;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
@@ -1059,7 +1105,7 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
         prefetch_tmap(&p.tm_vg);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -1070,9 +1116,9 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
     // The set-up above may overlap the prep kernel; each role waits for it
     // (griddepcontrol.wait) before it reads prep's output.
     if (warp == 0) {
-        if (lane == 0) producer_role(p, smem, bars, abort_flag);
+        if (lane == 0) producer_role<HD>(p, smem, bars, abort_flag);
     } else if (warp == 1) {
-        if (lane == 0) mma_role<kHalf>(p, smem, bars, abort_flag, tmem_base);
+        if (lane == 0) mma_role<kHalf, HD>(p, smem, bars, abort_flag, tmem_base);
     } else {
         {  // touch every 64-byte line of the parameters once, so the producer's walk hits in cache
             const int t = threadIdx.x - 64;
@@ -1083,7 +1129,7 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
                 asm volatile("" ::"r"(v));
             }
         }
-        softmax_role<kSearch, kHalf>(p, smem, bars, abort_flag, tmem_base);
+        softmax_role<kSearch, kHalf, HD>(p, smem, bars, abort_flag, tmem_base);
     }
 
     tc_fence_before();
@@ -1094,7 +1140,7 @@ __global__ void __launch_bounds__(kBandThreads, kBandCtasPerSm) band_tc_kernel(c
     if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, kStatusTimeout);
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 

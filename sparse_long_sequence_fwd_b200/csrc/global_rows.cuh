@@ -26,6 +26,10 @@ template <>
 __device__ __forceinline__ float load_as_float<__nv_bfloat16>(const __nv_bfloat16* p) {
     return __bfloat162float(*p);
 }
+template <>
+__device__ __forceinline__ float load_as_float<__half>(const __half* p) {
+    return __half2float(*p);
+}
 
 template <typename Tin>
 __device__ __forceinline__ void store_from_float(Tin* p, float x);
@@ -34,6 +38,10 @@ __device__ __forceinline__ void store_from_float<float>(float* p, float x) { *p 
 template <>
 __device__ __forceinline__ void store_from_float<__nv_bfloat16>(__nv_bfloat16* p, float x) {
     *p = __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ void store_from_float<__half>(__half* p, float x) {
+    *p = __float2half_rn(x);
 }
 
 __device__ __forceinline__ float block_reduce_max(float v, float* red) {

@@ -66,6 +66,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // GPUs run it on 296 CTAs too), so its partial-state region has a size
 // known without a device.
 constexpr int kMaxBandCtas = 296;
+// ... for a head dimension (one CTA per SM at HD = 128)
+constexpr int max_band_ctas(int d) { return d == 64 ? kMaxBandCtas : kMaxBandCtas / 2; }
 
 struct Layout {
     size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, off_qg, off_bcnt, off_bpart,
@@ -79,7 +81,7 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
     Layout L{};
     L.W = (T + 31) / 32;
     L.gstride = std::max(1, std::min(n_global, T));
-    if (dtype != LF_F32) {
+    if (dtype != LF_F32 && d == 64) {
         // tensor-core global rows: 128-key chunks, cpc per CTA, about three CTAs
         // per SM of a 148-SM B200 (each holds a two-stage ring of 72 KB)
         const int nblk = (T + kGrKeys - 1) / kGrKeys;
@@ -116,7 +118,7 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
     L.off_vg = o;
     L.off_qg = o;
     if (dtype != LF_F32 && n_global > 0) {
-        const size_t kgb = sizeof(__nv_bfloat16) * size_t(B) * H * L.ngp * 64;
+        const size_t kgb = sizeof(__nv_bfloat16) * size_t(B) * H * L.ngp * d;
         L.off_vg = align256(o + kgb);
         L.off_qg = align256(L.off_vg + kgb);
         o = align256(L.off_qg + kgb);
@@ -128,7 +130,8 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
         // every head has at most ceil(T / 128) + kMaxDilTma - 1 tiles (one per residue class more)
         L.band_tiles = (long long)B * H * ((T + kBM - 1) / kBM + kMaxDilTma - 1);
         L.off_bpart = align256(o + sizeof(int32_t) * size_t(L.band_tiles) * 8);
-        o = align256(L.off_bpart + sizeof(float) * size_t(2 * kMaxBandCtas) * kPartFloats);
+        const size_t part_floats = d == 64 ? BandCfg<64>::kPartFloats : BandCfg<128>::kPartFloats;
+        o = align256(L.off_bpart + sizeof(float) * size_t(2 * max_band_ctas(d)) * part_floats);
     }
     L.total = std::max<size_t>(o, 256);
     return L;
@@ -145,9 +148,17 @@ bool is_capturing(cudaStream_t s) {
 lf_status set_kernel_attributes() {
     const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + 2 * kMaxGlobal) * 4;
     const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
-    for (auto kern : {band_tc_kernel<false, false>, band_tc_kernel<true, false>, band_tc_kernel<false, true>,
-                      band_tc_kernel<true, true>})
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBandSmem) != cudaSuccess ||
+    for (auto kern : {band_tc_kernel<false, false, 64>, band_tc_kernel<true, false, 64>,
+                      band_tc_kernel<false, true, 64>, band_tc_kernel<true, true, 64>})
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BandCfg<64>::kSmem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+            return LF_ERR_CUDA;
+    for (auto kern : {band_tc_kernel<false, false, 128>, band_tc_kernel<true, false, 128>,
+                      band_tc_kernel<false, true, 128>, band_tc_kernel<true, true, 128>})
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BandCfg<128>::kSmem) !=
+                cudaSuccess ||
             cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return LF_ERR_CUDA;
@@ -162,6 +173,10 @@ lf_status set_kernel_attributes() {
         cudaFuncSetAttribute(global_rows_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
             cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_kernel<__nv_bfloat16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gr_max) != cudaSuccess ||
+        cudaFuncSetAttribute(global_rows_kernel<__half, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
             cudaSuccess)
         return LF_ERR_CUDA;
     return LF_OK;
@@ -225,13 +240,14 @@ lf_status get_encoder() {
     return LF_OK;
 }
 
-// 3-D map of 16-bit elements (bf16, or f16 when half) over [d=64, rows, B*H]
-// with a 128-byte swizzle; box = 64 x (rows_per_box * stride) x 1, element
-// stride `stride` along the rows.
+// 3-D map of 16-bit elements (bf16, or f16 when half) over [d, rows, B*H]
+// (d = 64 or 128) with a 128-byte swizzle; box = 64 x (rows_per_box *
+// stride) x 1 (one 64-column sub-tile; with d = 128 two boxes per row, at
+// x = 0 and 64), element stride `stride` along the rows.
 lf_status encode_rows_map(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t bh, uint32_t rows_per_box,
-                          uint32_t stride, bool half) {
-    cuuint64_t gdim[3] = {64, rows, bh};
-    cuuint64_t gstr[2] = {64 * 2, rows * 64 * 2};
+                          uint32_t stride, bool half, int d) {
+    cuuint64_t gdim[3] = {static_cast<cuuint64_t>(d), rows, bh};
+    cuuint64_t gstr[2] = {static_cast<cuuint64_t>(d) * 2, rows * d * 2};
     cuuint32_t box[3] = {64, rows_per_box * stride, 1};
     cuuint32_t estr[3] = {1, stride, 1};
     CUresult r = g_encode(tm, half ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstr, box, estr,
@@ -261,7 +277,7 @@ lf_status check_args(const void* q, const void* k, const void* v, void* out, int
     if (dtype == LF_F32 && d > 128) return LF_ERR_UNSUPPORTED;
     if (n_global > 0 && uint64_t(B) * H > 65535u) return LF_ERR_UNSUPPORTED;  // global-row grid.y
     if (dtype != LF_F32) {  // the tensor-core path, bf16 or f16
-        if (d != 64 || H > kMaxHeads) return LF_ERR_UNSUPPORTED;
+        if ((d != 64 && d != 128) || H > kMaxHeads) return LF_ERR_UNSUPPORTED;
         int kinds[kMaxDilKinds];
         int nk = 0;
         for (int h = 0; h < H; ++h) {
@@ -440,9 +456,9 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         for (int kd = 0; kd < nk; ++kd) {
             const int dl = bp.dk_dil[kd];
             const uint32_t R = static_cast<uint32_t>(bp.dk_rows[kd]);
-            if ((st = encode_rows_map(&bp.tm_q[kd], q, T, uint64_t(B) * H, R, dl, half)) != LF_OK ||
-                (st = encode_rows_map(&bp.tm_k[kd], k, T, uint64_t(B) * H, R, dl, half)) != LF_OK ||
-                (st = encode_rows_map(&bp.tm_v[kd], v, T, uint64_t(B) * H, R, dl, half)) != LF_OK)
+            if ((st = encode_rows_map(&bp.tm_q[kd], q, T, uint64_t(B) * H, R, dl, half, d)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_k[kd], k, T, uint64_t(B) * H, R, dl, half, d)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_v[kd], v, T, uint64_t(B) * H, R, dl, half, d)) != LF_OK)
                 return st;
         }
         for (int a = nk; a < kMaxDilKinds; ++a) {  // unused slots: valid maps, never read
@@ -451,15 +467,17 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
             bp.tm_v[a] = bp.tm_v[0];
         }
         if (n_global > 0) {
-            if ((st = encode_rows_map(&bp.tm_kg, ws.kg, L.ngp, uint64_t(B) * H, kBN, 1, half)) != LF_OK ||
-                (st = encode_rows_map(&bp.tm_vg, ws.vg, L.ngp, uint64_t(B) * H, kBN, 1, half)) != LF_OK)
+            if ((st = encode_rows_map(&bp.tm_kg, ws.kg, L.ngp, uint64_t(B) * H, kBN, 1, half, d)) != LF_OK ||
+                (st = encode_rows_map(&bp.tm_vg, ws.vg, L.ngp, uint64_t(B) * H, kBN, 1, half, d)) != LF_OK)
                 return st;
         } else {
             bp.tm_kg = bp.tm_k[0];
             bp.tm_vg = bp.tm_v[0];
         }
         if ((st = band_schedule(bp, B, H, T, r_eff, n_global > 0 ? (L.gstride + kBN - 1) / kBN : 0, kind_of_head,
-                                std::min(kBandCtasPerSm * ds->sm_count, kMaxBandCtas), L.band_tiles)) != LF_OK)
+                                std::min((d == 64 ? BandCfg<64>::kCtasPerSm : BandCfg<128>::kCtasPerSm) * ds->sm_count,
+                                         max_band_ctas(d)),
+                                L.band_tiles)) != LF_OK)
             return st;
         bp.cnt = reinterpret_cast<int32_t*>(base + L.off_bcnt);
         bp.part = reinterpret_cast<float*>(base + L.off_bpart);
@@ -476,13 +494,13 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         const unsigned long long wl = g_test_wait_ns.load();
         bp.wait_ns = wl ? wl : LF_WAIT_NS;
         bp.test_stall = g_test_stall.load();
-        const int grid = bp.grid_ctas;  // persistent: two CTAs per SM
+        const int grid = bp.grid_ctas;  // persistent: two CTAs per SM (one at d = 128)
         // right after prep on the same stream, launched as its programmatic dependent: the
         // band kernel's set-up (barriers, TMEM, tensor-map prefetch) overlaps prep
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(grid));
         cfg.blockDim = dim3(kBandThreads);
-        cfg.dynamicSmemBytes = kBandSmem;
+        cfg.dynamicSmemBytes = d == 64 ? BandCfg<64>::kSmem : BandCfg<128>::kSmem;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -491,8 +509,10 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         cfg.numAttrs = 1;
         // more than 32 global tokens: the instantiation whose global-key dedup searches
         void (*kern)(BandTcParams) =
-            n_global > 32 ? (half ? band_tc_kernel<true, true> : band_tc_kernel<true, false>)
-                          : (half ? band_tc_kernel<false, true> : band_tc_kernel<false, false>);
+            d == 64 ? (n_global > 32 ? (half ? band_tc_kernel<true, true, 64> : band_tc_kernel<true, false, 64>)
+                                     : (half ? band_tc_kernel<false, true, 64> : band_tc_kernel<false, false, 64>))
+                    : (n_global > 32 ? (half ? band_tc_kernel<true, true, 128> : band_tc_kernel<true, false, 128>)
+                                     : (half ? band_tc_kernel<false, true, 128> : band_tc_kernel<false, false, 128>));
         if (cudaLaunchKernelEx(&cfg, kern, bp) != cudaSuccess) return LF_ERR_CUDA;
         ++launches;
     }
@@ -517,7 +537,15 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         gp.sl2 = sl2;
         gp.cpc = L.cpc;
         gp.ngp = L.ngp;
-        if (dtype != LF_F32) {
+        if (dtype != LF_F32 && d == 128) {
+            // 16-bit inputs with d = 128: the CUDA-core global-row kernel (chunks of keys, the
+            // last chunk of a (b, h) merges)
+            const dim3 grid(L.nchunk, B * H);
+            const size_t smem = size_t(kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
+            if (half) global_rows_kernel<__half, 128><<<grid, kGrThreads, smem, gs>>>(gp);
+            else global_rows_kernel<__nv_bfloat16, 128><<<grid, kGrThreads, smem, gs>>>(gp);
+            ++launches;
+        } else if (dtype != LF_F32) {
             // key splits x (b, h) x groups of kpw / 2 global rows, then the merge of the splits
             const int kpw = L.gr_kpw, rows = kpw / 2;
             const dim3 grid(L.nchunk, B * H, (L.gstride + rows - 1) / rows);

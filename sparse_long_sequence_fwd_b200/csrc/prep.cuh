@@ -153,22 +153,24 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     if (p.pack) {
         const int nk = n_k_total, nq = n_q_total;
         const size_t bh = static_cast<size_t>(b) * p.H + h;
-        const uint4* q4 = reinterpret_cast<const uint4*>(p.q) + bh * T * 8;
-        const uint4* k4 = reinterpret_cast<const uint4*>(p.k) + bh * T * 8;
-        const uint4* v4 = reinterpret_cast<const uint4*>(p.v) + bh * T * 8;
-        uint4* qg4 = reinterpret_cast<uint4*>(p.ws.qg) + bh * p.ngp * 8;
-        uint4* kg4 = reinterpret_cast<uint4*>(p.ws.kg) + bh * p.ngp * 8;
-        uint4* vg4 = reinterpret_cast<uint4*>(p.ws.vg) + bh * p.ngp * 8;
+        // 16-byte words per row: 8 (d = 64) or 16 (d = 128)
+        const int wsh = p.d == 128 ? 4 : 3, rw = 1 << wsh;
+        const uint4* q4 = reinterpret_cast<const uint4*>(p.q) + bh * T * rw;
+        const uint4* k4 = reinterpret_cast<const uint4*>(p.k) + bh * T * rw;
+        const uint4* v4 = reinterpret_cast<const uint4*>(p.v) + bh * T * rw;
+        uint4* qg4 = reinterpret_cast<uint4*>(p.ws.qg) + bh * p.ngp * rw;
+        uint4* kg4 = reinterpret_cast<uint4*>(p.ws.kg) + bh * p.ngp * rw;
+        uint4* vg4 = reinterpret_cast<uint4*>(p.ws.vg) + bh * p.ngp * rw;
 #pragma unroll 4
-        for (int idx = tid; idx < p.ngp * 8; idx += kPrepThreads) {  // (unrolled: the loads of several rows in flight)
-            int a = idx >> 3, c = idx & 7;
+        for (int idx = tid; idx < p.ngp * rw; idx += kPrepThreads) {  // (unrolled: the loads of several rows in flight)
+            int a = idx >> wsh, c = idx & (rw - 1);
             uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv, qv = kv;
             if (a < nk) {
                 size_t row = static_cast<size_t>(gk_s[a]);
-                kv = k4[row * 8 + c];
-                vv = v4[row * 8 + c];
+                kv = k4[row * rw + c];
+                vv = v4[row * rw + c];
             }
-            if (a < nq) qv = q4[static_cast<size_t>(gq_s[a]) * 8 + c];
+            if (a < nq) qv = q4[static_cast<size_t>(gq_s[a]) * rw + c];
             kg4[idx] = kv;
             vg4[idx] = vv;
             qg4[idx] = qv;

@@ -78,8 +78,11 @@ LARGE = Workload("large_T16384_g32", "bf16", 1, 16, 16384, 64, 256, _dil(16, 1),
 # the base workload with f16 inputs (the pages train with fp16 mixed
 # precision: Longformer wiki, section 6.3)
 BASE_F16 = dataclasses.replace(BASE, name="base_T4096_w513_f16", dtype="f16")
+# 128-dimensional heads (8 of them, the same model width as 16 heads of 64)
+D128 = Workload("d128_H8_T4096_w513", "bf16", 1, 8, 4096, 128, 256, _dil(8, 1),
+                globals_per_b=[[0]], scale=128 ** -0.5, seed=1006)
 
-ALL = [TINY, BASE, QA, DILATED, LARGE, BASE_F16]
+ALL = [TINY, BASE, QA, DILATED, LARGE, BASE_F16, D128]
 BY_NAME = {w.name: w for w in ALL}
 
 

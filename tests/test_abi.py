@@ -62,10 +62,10 @@ def _call(lib, **kw):
     (dict(q=P(FAKE + 2)), 1),                                                    # misaligned
     (dict(dil=(ctypes.c_int32 * 2)(1, 0)), 1),                                   # dilation < 1
     (dict(B=1 << 20, H=1 << 20, T=1 << 20), 1),                                  # size overflow
-    (dict(d=32), 2), (dict(d=128), 2),                                           # bf16 path: d == 64 only
+    (dict(d=32), 2), (dict(d=96), 2), (dict(d=256), 2),                          # bf16 path: d == 64 or 128
     (dict(dil=(ctypes.c_int32 * 2)(1, 9)), 2),                                   # TMA element stride <= 8
     (dict(T=(1 << 20) + 1), 2), (dict(H=129), 2), (dict(dtype=0, d=129), 2),
-    (dict(dtype=2, d=128), 2), (dict(dtype=2, dil=(ctypes.c_int32 * 2)(1, 9)), 2),  # f16: same limits as bf16
+    (dict(dtype=2, d=32), 2), (dict(dtype=2, dil=(ctypes.c_int32 * 2)(1, 9)), 2),  # f16: same limits as bf16
     (dict(dtype=3), 1),
 ])
 def test_argument_errors_return_status_without_launch(lib, kw, code):

@@ -248,13 +248,13 @@ def test_output_guard_regions_untouched():
     parity.compare(w, out, parity.oracle_full(w, inp))
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f16"])
-def test_host_entry_point_matches_device_entry_point(dtype):
+@pytest.mark.parametrize("dtype,d", [("bf16", 64), ("f16", 64), ("bf16", 128)])
+def test_host_entry_point_matches_device_entry_point(dtype, d):
     """The host entry point runs the call as slices of (sample, heads), one
     launch each, so the band kernel splits its work differently from one
     whole launch and split tiles merge in another order: both entry points
     are compared with the oracle, and with each other at the same bar."""
-    w = workloads.custom("host_api", dtype, 2, 2, 700, 64, 60, globals_per_b=[[0, 5], [9, 9]],
+    w = workloads.custom("host_api", dtype, 2, 2, 700, d, 60, globals_per_b=[[0, 5], [9, 9]],
                          pad_from=[None, 600], seed=42)
     inp = workloads.make_inputs(w)
     dev = parity.run_gpu(w, inp)
@@ -320,4 +320,23 @@ def test_f16_cases_full_case(w):
 @pytest.mark.parametrize("base", [workloads.BASE, workloads.QA], ids=lambda w: w.name)
 def test_f16_full_size_every_element(base):
     w = dataclasses.replace(base, name=base.name + "_f16", dtype="f16")
+    _full_case(w)
+
+
+# d = 128 heads on the tensor cores (one CTA per SM: O takes 128 TMEM columns)
+D128_CASES = [
+    workloads.custom("bf16_d128_multi_tile", "bf16", 2, 3, 1000, 128, 100, dil=[1, 2, 3],
+                     globals_per_b=[[0, 999, 500, 500], [7, 3, 3, 640]], pad_from=[None, 777], seed=61),
+    workloads.custom("f16_d128_multi_tile", "f16", 2, 3, 1000, 128, 100, dil=[1, 2, 3],
+                     globals_per_b=[[0, 999, 500, 500], [7, 3, 3, 640]], pad_from=[None, 777], seed=62),
+    workloads.custom("bf16_d128_49_globals_dil", "bf16", 2, 4, 1500, 128, 60, dil=[1, 2, 3, 4],
+                     globals_per_b=[list(range(5, 1500, 31)) + [5, 36], list(range(700, 1100, 9)) + [1096] * 6],
+                     pad_from=[1400, None], seed=63),
+    workloads.custom("bf16_d128_T4096_r256", "bf16", 1, 6, 4096, 128, 256, globals_per_b=[[0]], seed=64),
+    workloads.custom("f16_d128_T129_no_globals", "f16", 1, 2, 129, 128, 128, seed=65),
+]
+
+
+@pytest.mark.parametrize("w", D128_CASES, ids=lambda w: w.name)
+def test_d128_cases_every_element(w):
     _full_case(w)
