@@ -110,6 +110,37 @@ __device__ __forceinline__ void merge_partials(const GlobalRowParams& p, int bh,
     }
 }
 
+// The kChunk rows [chunk * kChunk, +kChunk) of a 16-bit [T][DP] matrix into
+// shared memory as fp32 (rows past T are zero): 16-byte loads, all of a
+// thread's loads issued before any is used, so the copy costs one round trip
+// to memory.  kSkew: element c of row jj goes to column (c + jj) mod DP.
+template <typename Tin, int DP, bool kSkew>
+__device__ __forceinline__ void stage_chunk16(float* dst, const Tin* src, int chunk, int T) {
+    constexpr int kVec = 8;                                  // elements per 16-byte word
+    constexpr int kRowWords = DP / kVec;
+    constexpr int kPer = kChunk * kRowWords / kGrThreads;    // words per thread
+    static_assert(kPer * kGrThreads == kChunk * kRowWords, "whole words per thread");
+    const int tid = threadIdx.x;
+    uint4 u[kPer];
+#pragma unroll
+    for (int it = 0; it < kPer; ++it) {
+        const int w = tid + it * kGrThreads, jj = w / kRowWords, c0 = (w - jj * kRowWords) * kVec;
+        const int jg = chunk * kChunk + jj;
+        u[it] = jg < T ? *reinterpret_cast<const uint4*>(src + static_cast<size_t>(jg) * DP + c0)
+                       : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int it = 0; it < kPer; ++it) {
+        const int w = tid + it * kGrThreads, jj = w / kRowWords, c0 = (w - jj * kRowWords) * kVec;
+        const Tin* e = reinterpret_cast<const Tin*>(&u[it]);
+#pragma unroll
+        for (int t = 0; t < kVec; ++t) {
+            const int c = c0 + t;
+            dst[jj * DP + (kSkew ? ((c + jj) & (DP - 1)) : c)] = load_as_float(e + t);
+        }
+    }
+}
+
 // DP: head dim rounded up to a multiple of 32 (32, 64 or 128).
 template <typename Tin, int DP>
 __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams p) {
@@ -135,16 +166,35 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
     const int j = chunk * kChunk + tid;
     const bool valid = j < T && !(p.pad && p.pad[static_cast<size_t>(b) * T + j]);
 
+    // the chunk's K rows, read coalesced into shared memory first (the V area;
+    // element c of row jj at column (c + jj) mod DP, so the row reads below
+    // hit 32 different banks), then each thread's row into registers
+    if constexpr (sizeof(Tin) == 2) {
+        stage_chunk16<Tin, DP, true>(vs, kb, chunk, T);  // (16-bit inputs: d == DP)
+    } else {
+        for (int idx = tid; idx < kChunk * DP; idx += kGrThreads) {
+            const int jj = idx / DP, c = idx - jj * DP;
+            const int jg = chunk * kChunk + jj;
+            vs[jj * DP + ((c + jj) & (DP - 1))] =
+                (jg < T && c < d) ? load_as_float(kb + static_cast<size_t>(jg) * d + c) : 0.f;
+        }
+    }
+    __syncthreads();
     float kr[DP];
 #pragma unroll
-    for (int c = 0; c < DP; ++c) kr[c] = (valid && c < d) ? load_as_float(kb + static_cast<size_t>(j) * d + c) : 0.f;
+    for (int c = 0; c < DP; ++c) kr[c] = valid ? vs[tid * DP + ((c + tid) & (DP - 1))] : 0.f;
+    __syncthreads();
     // V chunk into shared memory (coalesced), zero for invalid keys
-    for (int idx = tid; idx < kChunk * DP; idx += kGrThreads) {
-        int jj = idx / DP, c = idx - jj * DP;
-        int jg = chunk * kChunk + jj;
-        float x = 0.f;
-        if (jg < T && c < d) x = load_as_float(vb + static_cast<size_t>(jg) * d + c);
-        vs[idx] = x;
+    if constexpr (sizeof(Tin) == 2) {
+        stage_chunk16<Tin, DP, false>(vs, vb, chunk, T);
+    } else {
+        for (int idx = tid; idx < kChunk * DP; idx += kGrThreads) {
+            int jj = idx / DP, c = idx - jj * DP;
+            int jg = chunk * kChunk + jj;
+            float x = 0.f;
+            if (jg < T && c < d) x = load_as_float(vb + static_cast<size_t>(jg) * d + c);
+            vs[idx] = x;
+        }
     }
 
     const int groups = kGrThreads / DP;  // key groups for the p*v sum
