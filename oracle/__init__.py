@@ -43,6 +43,8 @@ def _load():
         lib.lf_oracle_rows.restype = I
         lib.lf_oracle_fwd.argtypes = [P, P, P, P, I, I, I, I, I, P, P, I, P, ctypes.c_double, I]
         lib.lf_oracle_fwd.restype = I
+        lib.lf_oracle_fwd_rand.argtypes = [P, P, P, P, I, I, I, I, I, P, P, I, P, ctypes.c_double, I, P, I]
+        lib.lf_oracle_fwd_rand.restype = I
         lib.lf_oracle_key_set.argtypes = [I, I, I, I, P, I, P, P]
         lib.lf_oracle_key_set.restype = I
         lib.lf_oracle_key_total.argtypes = [I, I, I, P, I, P]
@@ -92,8 +94,10 @@ def _dil(dil, H):
 
 
 def fwd(q, k, v, r: int, dil=None, global_idx=None, key_pad_mask=None, scale: float = None,
-        nthreads: int = 0) -> np.ndarray:
-    """All rows.  q, k, v: [B, H, T, d]; returns fp64 [B, H, T, d]."""
+        nthreads: int = 0, rand_blocks=None) -> np.ndarray:
+    """All rows.  q, k, v: [B, H, T, d]; returns fp64 [B, H, T, d].
+    rand_blocks (the BigBird variant): int [B, H, ceil(T / 64), n_rand], the
+    random key blocks of every 64-row query block (see lf_oracle.c)."""
     q, k, v = _f32(q), _f32(k), _f32(v)
     B, H, T, d = q.shape
     gi = _i32(global_idx)
@@ -103,8 +107,14 @@ def fwd(q, k, v, r: int, dil=None, global_idx=None, key_pad_mask=None, scale: fl
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     out = np.empty((B, H, T, d), dtype=np.float64)
-    st = _load().lf_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, d, int(r), _ptr(dl),
-                               _ptr(gi), n_global, _ptr(pad), float(scale), int(nthreads))
+    rb = _i32(rand_blocks)
+    n_rand = 0
+    if rb is not None:
+        assert rb.shape[:3] == (B, H, (T + 63) // 64), rb.shape
+        n_rand = rb.shape[3]
+    st = _load().lf_oracle_fwd_rand(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, d, int(r), _ptr(dl),
+                                    _ptr(gi), n_global, _ptr(pad), float(scale), int(nthreads),
+                                    _ptr(rb) if n_rand else None, n_rand)
     if st != 0:
         raise RuntimeError("oracle failed with status %d" % st)
     return out

@@ -31,6 +31,18 @@
  *       ("Longformer" note, the y_i equation and the "Mask View" section).
  *     * K(i) empty -> y_i = 0 (the pages are silent; this is the reading
  *       taken).
+ *     * Random blocks (the BigBird variant, lf_oracle_fwd_rand): an
+ *       ordinary row also keeps the keys of the random key blocks drawn for
+ *       its query block, K(i) U R(i), before padding is removed.  BigBird
+ *       adds random attention to the window and the global tokens, each
+ *       token attending a few randomly chosen others (mhpn.cn page, section
+ *       2.2.1), in blocks of block_size = 64 (same page, section 2.2.2; the
+ *       aiqz.cc page's BigBird comparison: neighbours + front desk + random
+ *       picks).  Reading taken: query block i / 64 draws n_rand key blocks
+ *       (passed in, since the draws are random); key block c holds keys
+ *       [64 c, 64 c + 64) clipped to T; blocks outside [0, ceil(T / 64))
+ *       are ignored; a set again, so duplicates and keys already in K(i)
+ *       count once.  Global rows are unchanged.
  *
  * Readings of points the pages leave open: 0-based indices; r is the
  * one-sided radius; the dilated window is {i + dil*t : |t| <= r} (the
@@ -53,6 +65,7 @@
 #endif
 
 #define OR_OK 0
+#define OR_RAND_BLOCK 64  /* BigBird block_size */
 #define OR_BAD_ARG 1
 #define OR_NO_MEM 4
 
@@ -69,7 +82,7 @@ static int is_global(int i, int T, const int32_t* G, int nG)
  * its size.  `marker` is caller scratch of T bytes.
  */
 static int key_set(int T, int r, int dil, int i, const int32_t* G, int nG,
-                   const uint8_t* pad_b, uint8_t* marker, int* keys)
+                   const uint8_t* pad_b, const int32_t* rnd, int n_rand, uint8_t* marker, int* keys)
 {
     memset(marker, 0, (size_t)T);
     if (is_global(i, T, G, nG)) {
@@ -81,6 +94,14 @@ static int key_set(int T, int r, int dil, int i, const int32_t* G, int nG,
         }
         for (int a = 0; a < nG; a++)
             if (G[a] >= 0 && G[a] < T) marker[G[a]] = 1;
+        if (rnd) {  /* rnd: [ceil(T / 64)][n_rand] key blocks of each query block of this (b, h) */
+            const int32_t* ri = rnd + (size_t)(i / OR_RAND_BLOCK) * n_rand;
+            for (int a = 0; a < n_rand; a++) {
+                long j0 = (long)ri[a] * OR_RAND_BLOCK;
+                if (ri[a] < 0 || j0 >= T) continue;
+                for (long j = j0; j < j0 + OR_RAND_BLOCK && j < T; j++) marker[j] = 1;
+            }
+        }
     }
     if (pad_b)
         for (int j = 0; j < T; j++)
@@ -95,10 +116,10 @@ static int key_set(int T, int r, int dil, int i, const int32_t* G, int nG,
  * softmax weights p_j / l at the key positions and 0 elsewhere. */
 static void one_row(const float* q, const float* k, const float* v, double* y,
                     int T, int d, int r, int dil, int i, const int32_t* G, int nG,
-                    const uint8_t* pad_b, double scale,
+                    const uint8_t* pad_b, const int32_t* rnd, int n_rand, double scale,
                     uint8_t* marker, int* keys, double* s, double* probs)
 {
-    int n = key_set(T, r, dil, i, G, nG, pad_b, marker, keys);
+    int n = key_set(T, r, dil, i, G, nG, pad_b, rnd, n_rand, marker, keys);
     if (probs)
         for (int j = 0; j < T; j++) probs[j] = 0.0;
     if (n == 0) {
@@ -142,14 +163,16 @@ static int check_args(int B, int H, int T, int d, int r, const int32_t* dil, int
  * when n_global == 0).  key_pad: uint8 [B, T] or NULL.  nthreads <= 0 uses
  * the OpenMP default.
  */
-int lf_oracle_rows(const float* q, const float* k, const float* v,
-                   int B, int H, int T, int d, int r, const int32_t* dil,
-                   const int32_t* global_idx, int n_global, const uint8_t* key_pad,
-                   double scale, const int32_t* rows, long n_rows, double* out_rows,
-                   int nthreads)
+int lf_oracle_rows_rand(const float* q, const float* k, const float* v,
+                        int B, int H, int T, int d, int r, const int32_t* dil,
+                        const int32_t* global_idx, int n_global, const uint8_t* key_pad,
+                        double scale, const int32_t* rows, long n_rows, double* out_rows,
+                        int nthreads, const int32_t* rand_blocks, int n_rand)
 {
     int st = check_args(B, H, T, d, r, dil, n_global);
     if (st) return st;
+    if (n_rand < 0 || (n_rand > 0 && !rand_blocks)) return OR_BAD_ARG;
+    const long nqb = (T + OR_RAND_BLOCK - 1) / OR_RAND_BLOCK;
     for (long n = 0; n < n_rows; n++) {
         int b = rows[3 * n], h = rows[3 * n + 1], i = rows[3 * n + 2];
         if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= T) return OR_BAD_ARG;
@@ -175,8 +198,9 @@ int lf_oracle_rows(const float* q, const float* k, const float* v,
                 size_t bh = (size_t)b * H + h;
                 const int32_t* G = n_global > 0 ? global_idx + (size_t)b * n_global : NULL;
                 const uint8_t* pad_b = key_pad ? key_pad + (size_t)b * T : NULL;
+                const int32_t* rnd = n_rand > 0 ? rand_blocks + bh * (size_t)nqb * n_rand : NULL;
                 one_row(q + bh * T * d, k + bh * T * d, v + bh * T * d, out_rows + (size_t)n * d,
-                        T, d, r, dil[h], i, G, n_global, pad_b, scale, marker, keys, s, NULL);
+                        T, d, r, dil[h], i, G, n_global, pad_b, rnd, n_rand, scale, marker, keys, s, NULL);
             }
         }
         free(marker);
@@ -186,11 +210,22 @@ int lf_oracle_rows(const float* q, const float* k, const float* v,
     return err ? OR_NO_MEM : OR_OK;
 }
 
-/* Every row: out is double [B, H, T, d]. */
-int lf_oracle_fwd(const float* q, const float* k, const float* v, double* out,
-                  int B, int H, int T, int d, int r, const int32_t* dil,
-                  const int32_t* global_idx, int n_global, const uint8_t* key_pad,
-                  double scale, int nthreads)
+int lf_oracle_rows(const float* q, const float* k, const float* v,
+                   int B, int H, int T, int d, int r, const int32_t* dil,
+                   const int32_t* global_idx, int n_global, const uint8_t* key_pad,
+                   double scale, const int32_t* rows, long n_rows, double* out_rows,
+                   int nthreads)
+{
+    return lf_oracle_rows_rand(q, k, v, B, H, T, d, r, dil, global_idx, n_global, key_pad, scale,
+                               rows, n_rows, out_rows, nthreads, NULL, 0);
+}
+
+/* Every row: out is double [B, H, T, d].  rand_blocks: int32
+ * [B, H, ceil(T / 64), n_rand] (NULL when n_rand == 0). */
+int lf_oracle_fwd_rand(const float* q, const float* k, const float* v, double* out,
+                       int B, int H, int T, int d, int r, const int32_t* dil,
+                       const int32_t* global_idx, int n_global, const uint8_t* key_pad,
+                       double scale, int nthreads, const int32_t* rand_blocks, int n_rand)
 {
     int st = check_args(B, H, T, d, r, dil, n_global);
     if (st) return st;
@@ -206,10 +241,19 @@ int lf_oracle_fwd(const float* q, const float* k, const float* v, double* out,
                 rows[3 * n + 2] = i;
                 n++;
             }
-    st = lf_oracle_rows(q, k, v, B, H, T, d, r, dil, global_idx, n_global, key_pad, scale,
-                        rows, n_rows, out, nthreads);
+    st = lf_oracle_rows_rand(q, k, v, B, H, T, d, r, dil, global_idx, n_global, key_pad, scale,
+                             rows, n_rows, out, nthreads, rand_blocks, n_rand);
     free(rows);
     return st;
+}
+
+int lf_oracle_fwd(const float* q, const float* k, const float* v, double* out,
+                  int B, int H, int T, int d, int r, const int32_t* dil,
+                  const int32_t* global_idx, int n_global, const uint8_t* key_pad,
+                  double scale, int nthreads)
+{
+    return lf_oracle_fwd_rand(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, key_pad, scale,
+                              nthreads, NULL, 0);
 }
 
 /* K(i) of one row of sample b (head dilation `dil`): writes the sorted keys,
@@ -225,7 +269,7 @@ int lf_oracle_key_set(int T, int r, int dil, int i, const int32_t* G, int nG,
         free(keys);
         return -1;
     }
-    int n = key_set(T, r, dil, i, G, nG, pad_b, marker, keys);
+    int n = key_set(T, r, dil, i, G, nG, pad_b, NULL, 0, marker, keys);
     if (keys_out)
         for (int a = 0; a < n; a++) keys_out[a] = keys[a];
     free(marker);
@@ -245,7 +289,7 @@ long lf_oracle_key_total(int T, int r, int dil, const int32_t* G, int nG, const 
         return -1;
     }
     long total = 0;
-    for (int i = 0; i < T; i++) total += key_set(T, r, dil, i, G, nG, pad_b, marker, keys);
+    for (int i = 0; i < T; i++) total += key_set(T, r, dil, i, G, nG, pad_b, NULL, 0, marker, keys);
     free(marker);
     free(keys);
     return total;
@@ -274,7 +318,7 @@ int lf_oracle_row_probs(const float* q, const float* k, const float* v,
     const int32_t* G = n_global > 0 ? global_idx + (size_t)b * n_global : NULL;
     const uint8_t* pad_b = key_pad ? key_pad + (size_t)b * T : NULL;
     one_row(q + bh * T * d, k + bh * T * d, v + bh * T * d, y, T, d, r, dil[h], i, G, n_global,
-            pad_b, scale, marker, keys, s, probs);
+            pad_b, NULL, 0, scale, marker, keys, s, probs);
     free(marker);
     free(keys);
     free(s);
