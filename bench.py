@@ -59,7 +59,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-others", action="store_true",
-                    help="skip the QA, dilated, large, f16 base and d = 128 workload entries")
+                    help="skip the QA, dilated, large, f16 base, d = 128 and BigBird workload entries")
     return ap.parse_args()
 
 
@@ -109,6 +109,8 @@ def split_flops(w, inp):
         n_gq = int((~keep[b]).sum())
         for h in range(w.H):
             cnt = flops_mod.row_key_counts(w.T, w.r, int(w.dil[h]), Gb, pb)
+            if inp.get("rand_blocks") is not None:  # the BigBird variant's random keys
+                cnt = cnt + flops_mod.rand_extra_counts(w.T, w.r, Gb, pb, inp["rand_blocks"][b, h].numpy())
             total += int(cnt.sum())
             band += int(cnt[keep[b]].sum())
             if n_gq:
@@ -214,6 +216,7 @@ class WorkloadRun:
             self.sets.append((q0.clone(), k0.clone(), v0.clone(), torch.empty_like(q0)))
         self.gidx = inp["global_idx"].to(dev) if inp["global_idx"] is not None else None
         self.pad = inp["key_pad_mask"].to(dev) if inp["key_pad_mask"] is not None else None
+        self.rnd = inp["rand_blocks"].to(dev) if inp.get("rand_blocks") is not None else None
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             for i in range(max(warmup, 0)):
@@ -224,7 +227,8 @@ class WorkloadRun:
     def call(self, i, stages=7):
         q, k, v, o = self.sets[i % self.n_sets]
         self.lf_attn.fwd(q, k, v, self.w.r, dil=self.inp["dil"], global_idx=self.gidx, key_pad_mask=self.pad,
-                         scale=self.w.softmax_scale, out=o, stages=stages, stream=self.stream)
+                         scale=self.w.softmax_scale, out=o, stages=stages, stream=self.stream,
+                         rand_blocks=self.rnd)
 
     def capture(self, n, stages=7):
         g = self.torch.cuda.CUDAGraph()
@@ -274,14 +278,19 @@ class WorkloadRun:
 
     def summary(self, ms_per_step, peaks, world=1):
         w = self.w
-        band_us = self.stage_us(2)
         out = {"value": round(sharding.job_rate(self.total_f, world, ms_per_step * 1e-3) / 1e12, 3),
                "unit": "TFLOP/s", "ms_per_step": round(ms_per_step, 6),
                "tokens_per_s": round(sharding.job_rate(w.B * w.T, world, ms_per_step * 1e-3), 1),
-               "useful_gflop_per_step": round(self.total_f / 1e9, 4),
-               "band_tc_us": round(band_us, 2),
+               "useful_gflop_per_step": round(self.total_f / 1e9, 4)}
+        if self.rnd is not None:  # the per-stage entry point has no random-block form: the step only
+            out["stages"] = "not timed separately (random key blocks)"
+            out["l2"] = "rotating %d input sets, %.0f MB > 2x L2 (%.0f MB)" % (
+                self.n_sets, self.n_sets * self.set_bytes / 1e6, self.l2 / 1e6)
+            return out
+        band_us = self.stage_us(2)
+        out.update({"band_tc_us": round(band_us, 2),
                "band_frac": round(self.band_f / (band_us * 1e-6) / 1e12 / peaks["bf16_tflops"], 4),
-               "prep_us": round(self.stage_us(1), 2)}
+               "prep_us": round(self.stage_us(1), 2)})
         if self.gidx is not None:
             gr_us = self.stage_us(4)
             out["global_rows_us"] = round(gr_us, 2)
@@ -396,7 +405,7 @@ def run_ours(args):
     others = {}
     if rank == 0 and world == 1 and not args.no_others:
         for name in ("qa_B2_T4096_g64_pad", "dilated_T8192_r128", "large_T16384_g32", "base_T4096_w513_f16",
-                     "d128_H8_T4096_w513"):
+                     "d128_H8_T4096_w513", "bigbird_T4096_w513_rand3"):
             if name == w.name:
                 continue
             ow = workloads.BY_NAME[name]

@@ -113,6 +113,32 @@ lf_status lf_attn_fwd_host(const void* q, const void* k, const void* v, void* ou
                            void* stream);
 
 /*
+ * lf_attn_fwd_rand -- the BigBird variant: window + global tokens + random
+ * key blocks (the mhpn.cn page, sections 2.2.1 and 2.2.2: random attention
+ * beside the window and the global tokens, in blocks of 64; the aiqz.cc
+ * page's BigBird comparison).  Arguments as lf_attn_fwd, plus
+ *
+ *   rand_blocks DEVICE int32 [B, H, ceil(T / 64), n_rand]: the key blocks
+ *               drawn for each 64-row query block (key block c = keys
+ *               [64 c, 64 c + 64) clipped to T).  The caller draws them (for
+ *               instance from a seeded generator); entries outside
+ *               [0, ceil(T / 64)) are ignored.  NULL iff n_rand == 0.
+ *   n_rand      0..4 draws per query block.
+ *
+ *   An ordinary row i keeps K(i) of lf_attn_fwd together with the keys of
+ *   the blocks drawn for its query block i / 64, as a set (duplicate draws,
+ *   and keys already in the window or global, count once), padded keys
+ *   removed.  Global rows are unchanged.  n_rand == 0 is lf_attn_fwd.
+ *   With n_rand > 0: LF_BF16 or LF_F16, d == 64, every dil[h] == 1 (else
+ *   LF_ERR_UNSUPPORTED).
+ */
+lf_status lf_attn_fwd_rand(const void* q, const void* k, const void* v, void* out,
+                           int B, int H, int T, int d, int r, const int32_t* dil,
+                           const int32_t* global_idx, int n_global,
+                           const uint8_t* key_pad_mask, float scale, lf_dtype dtype,
+                           const int32_t* rand_blocks, int n_rand, void* stream);
+
+/*
  * lf_attn_fwd_stages -- runs a subset of the kernels lf_attn_fwd queues, for
  * timing one kernel at a time.  Same arguments as lf_attn_fwd, plus
  * stage_mask: bit 0 = prep (global lists, padding, packed global keys),

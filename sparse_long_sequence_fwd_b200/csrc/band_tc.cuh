@@ -73,6 +73,7 @@ constexpr int kBarQFull = 0, kBarQEmpty = kBarQFull + kQStages, kBarKFull = kBar
               kBarBufFree = kBarPFull + kSBufs, kBarOFull = kBarBufFree + kSBufs, kBarDrain = kBarOFull + 2,
               kNumBars = kBarDrain + 1;
 constexpr int kDescBytes = 128;
+constexpr int kMaxRand = 4;  // random key blocks per 64-row query block (the BigBird variant)
 constexpr int kMiscBytes = 16;
 constexpr uint32_t kColO = 192;
 
@@ -126,6 +127,7 @@ struct BandPiece {
     int s0, s1;        // the CTAs whose ranges hold the tile's blocks
     int last;          // 1: the last piece this CTA processes
     int tstart;        // position of the tile's first block in the sequence
+    int rb[2 * kMaxRand];  // random variant: the tile's random key blocks (-1: none), query block 0's then 1's
 };
 static_assert(sizeof(BandPiece) <= kDescBytes, "piece descriptor slot");
 
@@ -298,10 +300,11 @@ __device__ __forceinline__ float min32(const uint32_t* v) {
 // Only the global-key blocks read the prep kernel's output (packed keys), so
 // the wait for prep comes just before the first of them: the band blocks of
 // the first tile overlap prep.
-template <int HD>
+template <int HD, bool kRand>
 __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                               volatile int* abort_flag) {
     using C = BandCfg<HD>;
+    const int nrb = kRand ? p.nrb : 0;  // random key blocks per tile (dilation 1 only)
     const int s = blockIdx.x;
     const int x0 = range_start(p, s);
     const int x1 = range_start(p, s + 1);
@@ -330,6 +333,15 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
             for (int sub = 0; sub < C::kSub; ++sub)
                 for (int u = 0; u < kBN; u += d.R)
                     tma_load_3d(dst + sub * C::kKVSubBytes + u * 128, tm, full, 64 * sub, d.c + d.dil * (j0 + u), d.bh);
+        } else if (kRand && blk < d.nbb + nrb) {  // a random key block (none: rows past T, zero-filled)
+            mbar_arrive_expect_tx(full, C::kKVBytes);
+            const int rb = d.rb[blk - d.nbb];
+            const int j0 = rb >= 0 ? kBN * rb : p.T;
+            const CUtensorMap* tm = is_v ? &p.tm_v[d.dk] : &p.tm_k[d.dk];
+#pragma unroll
+            for (int sub = 0; sub < C::kSub; ++sub)
+                for (int u = 0; u < kBN; u += d.R)
+                    tma_load_3d(dst + sub * C::kKVSubBytes + u * 128, tm, full, 64 * sub, j0 + u, d.bh);
         } else {
             if (!prep_done) {  // packed global keys from here on
                 grid_dep_wait();
@@ -338,8 +350,8 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
             mbar_arrive_expect_tx(full, C::kKVBytes);
 #pragma unroll
             for (int sub = 0; sub < C::kSub; ++sub)
-                tma_load_3d(dst + sub * C::kKVSubBytes, is_v ? &p.tm_vg : &p.tm_kg, full, 64 * sub, (blk - d.nbb) * kBN,
-                            d.bh);
+                tma_load_3d(dst + sub * C::kKVSubBytes, is_v ? &p.tm_vg : &p.tm_kg, full, 64 * sub,
+                            (blk - d.nbb - nrb) * kBN, d.bh);
         }
         return true;
     };
@@ -388,6 +400,19 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
                 d.s1 = s1;
                 d.last = (!in_front && pend == x_main_end) ? 1 : 0;
                 d.tstart = cw->start;
+                if constexpr (kRand) {  // the draws of the tile's two query blocks (q0 / 64 and the next)
+                    const int nr = p.n_rand;
+#pragma unroll
+                    for (int k = 0; k < 2 * kMaxRand; ++k) {
+                        int rb = -1;
+                        if (k < 2 * nr) {
+                            const int qb = d.q0 / kBN + k / nr;
+                            if (qb < p.nqb) rb = p.rnd[(static_cast<size_t>(d.bh) * p.nqb + qb) * nr + k % nr];
+                            if (rb < 0 || rb >= p.nqb) rb = -1;  // outside the sequence: ignored
+                        }
+                        d.rb[k] = rb;
+                    }
+                }
                 *reinterpret_cast<BandPiece*>(smem + C::kOffDesc + qs * kDescBytes) = d;  // released by the arrive
                 mbar_arrive_expect_tx(&bars[kBarQFull + qs], C::kQBytes);
                 uint8_t* dQ = smem + C::kOffQ + qs * C::kQBytes;
@@ -446,10 +471,11 @@ __device__ __forceinline__ void producer_role(const BandTcParams& p, uint8_t* sm
 // With HD = 128, S sums the products of the two 64-column sub-tiles of Q and
 // K, and O's two 64-column halves each take the product with their own
 // sub-tile of V.
-template <bool kHalf, int HD>
+template <bool kHalf, int HD, bool kRand>
 __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                          volatile int* abort_flag, uint32_t tmem_base) {
     using C = BandCfg<HD>;
+    const int nrb = kRand ? p.nrb : 0;  // random key blocks per tile, after the band blocks
     const uint32_t idesc_pv = kHalf ? idesc_f16(kBM, 64, 0, 1) : idesc_bf16(kBM, 64, 0, 1);
     uint64_t dQ[kQStages];
 #pragma unroll
@@ -504,11 +530,11 @@ __device__ __forceinline__ void mma_role(const BandTcParams& p, uint8_t* smem, u
                 break;
             }
             tc_fence_after();
-            if (blk >= nbb && ngk < 0) {
+            if (blk >= nbb + nrb && ngk < 0) {
                 grid_dep_wait();
                 ngk = *reinterpret_cast<const volatile int*>(p.n_gk + bsm);
             }
-            const int ncols = blk < nbb ? kBN : global_block_cols(ngk, blk - nbb);
+            const int ncols = blk < nbb + nrb ? kBN : global_block_cols(ngk, blk - nbb - nrb);
             const uint32_t ids = kHalf ? idesc_f16(kBM, ncols, 0, 0) : idesc_bf16(kBM, ncols, 0, 0);
             const uint64_t dq = dQ[qs], dk = dK0 + kKVDescStep * st;
             const uint32_t tS = tmem_base + 64u * b;
@@ -772,7 +798,7 @@ __device__ __forceinline__ void flush_rows(const BandTcParams& p, const BandPiec
 
 // kSearch: the sample may have more than 32 global keys; the global-key block's
 // dedup then finds the keys in a row's window by binary search (below).
-template <bool kSearch, bool kHalf, int HD>
+template <bool kSearch, bool kHalf, int HD, bool kRand>
 __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* smem, uint64_t* bars,
                                              volatile int* abort_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -886,6 +912,32 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                             }
                             mk[c] = m;
                         }
+                    } else if (kRand && blk < nbb + p.nrb) {
+                        // a random key block of one of the tile's two query blocks: kept for the
+                        // rows of that query block, minus keys past T, in the row's window, global
+                        // (the global block has them) or padded, and minus a block its query
+                        // block drew before (a set: counted once)
+                        need_prep();  // the global-position bitmap
+                        const int k = blk - nbb, nr = p.n_rand, half = k / nr;
+                        const int rbk = dp->rb[k];
+                        bool dup = false;
+                        for (int kk = half * nr; kk < k; ++kk) dup |= dp->rb[kk] == rbk;
+                        const bool use = rbk >= 0 && !dup && (x >> 6) == half;  // the same for the whole warp
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            uint32_t m = 0u;
+                            const int j0 = kBN * rbk + 32 * c;
+                            if (use && j0 < p.T) {
+                                m = range_bits(0, p.T - j0) & ~range_bits(i - p.r - j0, i + p.r + 1 - j0);
+                                m &= ~p.gbit[static_cast<size_t>(dp->b) * p.W + (j0 >> 5)];
+                                if (p.pad) {
+                                    const int jd = j0 + lane;
+                                    const bool padded = jd < p.T && p.pad[static_cast<size_t>(dp->b) * p.T + jd] != 0;
+                                    m &= ~__ballot_sync(0xffffffffu, padded);
+                                }
+                            }
+                            mk[c] = m;
+                        }
                     } else {  // global keys not already in the row's window
                         const int bs = dp->b;
                         if (bs != gk_b) {
@@ -896,7 +948,7 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
                             gk_reg[0] = lane < ngk ? static_cast<uint32_t>(gl[lane]) : 0u;
                             gk_reg[1] = 32 + lane < ngk ? static_cast<uint32_t>(gl[32 + lane]) : 0u;
                         }
-                        const int gb = blk - nbb;
+                        const int gb = blk - nbb - (kRand ? p.nrb : 0);
                         const int nvalid = min(kBN, ngk - gb * kBN);
                         bool searched = false;
                         if constexpr (kSearch) {
@@ -1058,8 +1110,9 @@ __device__ __forceinline__ void softmax_role(const BandTcParams& p, uint8_t* sme
 // Instantiations from one source: kSearch = true for calls with more than 32
 // global tokens (see softmax_role), false otherwise, so each keeps its own
 // code for the block loop; kHalf = true for f16 inputs, false for bf16; HD =
-// the head dimension (64: two CTAs per SM; 128: one).
-template <bool kSearch, bool kHalf, int HD>
+// the head dimension (64: two CTAs per SM; 128: one); kRand: the BigBird
+// variant's random key blocks follow each tile's band blocks.
+template <bool kSearch, bool kHalf, int HD, bool kRand = false>
 __global__ void __launch_bounds__(kBandThreads, BandCfg<HD>::kCtasPerSm)
     band_tc_kernel(const __grid_constant__ BandTcParams p) {
     using C = BandCfg<HD>;
@@ -1116,9 +1169,9 @@ __global__ void __launch_bounds__(kBandThreads, BandCfg<HD>::kCtasPerSm)
     // The set-up above may overlap the prep kernel; each role waits for it
     // (griddepcontrol.wait) before it reads prep's output.
     if (warp == 0) {
-        if (lane == 0) producer_role<HD>(p, smem, bars, abort_flag);
+        if (lane == 0) producer_role<HD, kRand>(p, smem, bars, abort_flag);
     } else if (warp == 1) {
-        if (lane == 0) mma_role<kHalf, HD>(p, smem, bars, abort_flag, tmem_base);
+        if (lane == 0) mma_role<kHalf, HD, kRand>(p, smem, bars, abort_flag, tmem_base);
     } else {
         {  // touch every 64-byte line of the parameters once, so the producer's walk hits in cache
             const int t = threadIdx.x - 64;
@@ -1129,7 +1182,7 @@ __global__ void __launch_bounds__(kBandThreads, BandCfg<HD>::kCtasPerSm)
                 asm volatile("" ::"r"(v));
             }
         }
-        softmax_role<kSearch, kHalf, HD>(p, smem, bars, abort_flag, tmem_base);
+        softmax_role<kSearch, kHalf, HD, kRand>(p, smem, bars, abort_flag, tmem_base);
     }
 
     tc_fence_before();

@@ -149,7 +149,9 @@ lf_status set_kernel_attributes() {
     const int prep_max = (kMaxT / 32 + 2 * kPrepThreads + 2 * kMaxGlobal) * 4;
     const int gr_max = (kChunk * 128 + 128 + kChunk + 32 + kGrThreads) * 4;
     for (auto kern : {band_tc_kernel<false, false, 64>, band_tc_kernel<true, false, 64>,
-                      band_tc_kernel<false, true, 64>, band_tc_kernel<true, true, 64>})
+                      band_tc_kernel<false, true, 64>, band_tc_kernel<true, true, 64>,
+                      band_tc_kernel<false, false, 64, true>, band_tc_kernel<true, false, 64, true>,
+                      band_tc_kernel<false, true, 64, true>, band_tc_kernel<true, true, 64, true>})
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BandCfg<64>::kSmem) !=
                 cudaSuccess ||
             cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -372,7 +374,8 @@ lf_status band_schedule(BandTcParams& bp, int B, int H, int T, int r_eff, int ng
 
 lf_status launch_all(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d, int r,
                      const int32_t* dil, const int32_t* gidx, int n_global, const uint8_t* pad, float scale,
-                     lf_dtype dtype, cudaStream_t stream, DeviceState* ds, uint32_t stages = 7u) {
+                     lf_dtype dtype, cudaStream_t stream, DeviceState* ds, uint32_t stages = 7u,
+                     const int32_t* rnd = nullptr, int n_rand = 0) {
     const Layout L = make_layout(B, H, T, d, n_global, dtype);
     lf_status st = grow(&ds->ws, &ds->ws_bytes, L.total, stream);
     if (st != LF_OK) return st;
@@ -474,7 +477,14 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
             bp.tm_kg = bp.tm_k[0];
             bp.tm_vg = bp.tm_v[0];
         }
-        if ((st = band_schedule(bp, B, H, T, r_eff, n_global > 0 ? (L.gstride + kBN - 1) / kBN : 0, kind_of_head,
+        // after each tile's band blocks: 2 * n_rand random key blocks (the BigBird variant), then
+        // the global-key blocks
+        const int nrb = 2 * n_rand;
+        bp.rnd = rnd;
+        bp.n_rand = n_rand;
+        bp.nrb = nrb;
+        bp.nqb = (T + kBN - 1) / kBN;
+        if ((st = band_schedule(bp, B, H, T, r_eff, nrb + (n_global > 0 ? (L.gstride + kBN - 1) / kBN : 0), kind_of_head,
                                 std::min((d == 64 ? BandCfg<64>::kCtasPerSm : BandCfg<128>::kCtasPerSm) * ds->sm_count,
                                          max_band_ctas(d)),
                                 L.band_tiles)) != LF_OK)
@@ -509,10 +519,13 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         cfg.numAttrs = 1;
         // more than 32 global tokens: the instantiation whose global-key dedup searches
         void (*kern)(BandTcParams) =
-            d == 64 ? (n_global > 32 ? (half ? band_tc_kernel<true, true, 64> : band_tc_kernel<true, false, 64>)
-                                     : (half ? band_tc_kernel<false, true, 64> : band_tc_kernel<false, false, 64>))
-                    : (n_global > 32 ? (half ? band_tc_kernel<true, true, 128> : band_tc_kernel<true, false, 128>)
-                                     : (half ? band_tc_kernel<false, true, 128> : band_tc_kernel<false, false, 128>));
+            n_rand > 0  // (d == 64 only)
+                ? (n_global > 32 ? (half ? band_tc_kernel<true, true, 64, true> : band_tc_kernel<true, false, 64, true>)
+                                 : (half ? band_tc_kernel<false, true, 64, true> : band_tc_kernel<false, false, 64, true>))
+            : d == 64 ? (n_global > 32 ? (half ? band_tc_kernel<true, true, 64> : band_tc_kernel<true, false, 64>)
+                                       : (half ? band_tc_kernel<false, true, 64> : band_tc_kernel<false, false, 64>))
+                      : (n_global > 32 ? (half ? band_tc_kernel<true, true, 128> : band_tc_kernel<true, false, 128>)
+                                       : (half ? band_tc_kernel<false, true, 128> : band_tc_kernel<false, false, 128>));
         if (cudaLaunchKernelEx(&cfg, kern, bp) != cudaSuccess) return LF_ERR_CUDA;
         ++launches;
     }
@@ -642,6 +655,28 @@ lf_status lf_attn_fwd(const void* q, const void* k, const void* v, void* out, in
     if ((st = device_state(&ds)) != LF_OK) return st;
     return launch_all(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, key_pad_mask, scale, dtype,
                       static_cast<cudaStream_t>(stream), ds);
+}
+
+lf_status lf_attn_fwd_rand(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d,
+                           int r, const int32_t* dil, const int32_t* global_idx, int n_global,
+                           const uint8_t* key_pad_mask, float scale, lf_dtype dtype, const int32_t* rand_blocks,
+                           int n_rand, void* stream) {
+    lf_status st = check_args(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, scale, dtype);
+    if (st != LF_OK) return st;
+    if (n_rand < 0 || n_rand > kMaxRand || (n_rand > 0) != (rand_blocks != nullptr) ||
+        (reinterpret_cast<uintptr_t>(rand_blocks) & 3u))
+        return LF_ERR_INVALID_ARG;
+    if (n_rand > 0) {
+        if (dtype == LF_F32 || d != 64) return LF_ERR_UNSUPPORTED;
+        if (dil)
+            for (int h = 0; h < H; ++h)
+                if (dil[h] != 1) return LF_ERR_UNSUPPORTED;
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    if ((st = device_state(&ds)) != LF_OK) return st;
+    return launch_all(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, key_pad_mask, scale, dtype,
+                      static_cast<cudaStream_t>(stream), ds, 7u, rand_blocks, n_rand);
 }
 
 lf_status lf_attn_fwd_stages(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d,

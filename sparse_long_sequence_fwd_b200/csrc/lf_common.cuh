@@ -96,7 +96,12 @@ struct BandTcParams {
     int n_blocks;        // N (< 2^31)
     int grid_ctas;       // G
     int blk_q, blk_rm;   // N = blk_q * G + blk_rm
-    int blocks_per_b, tiles_per_b, ngb;
+    int blocks_per_b, tiles_per_b, ngb;  // ngb: blocks after the band blocks (random, then global keys)
+    // The BigBird variant (random key blocks): rnd [B*H][nqb][n_rand] key
+    // blocks of every 64-row query block; each tile's first nrb = 2 * n_rand
+    // blocks after its band blocks are its two query blocks' draws (0: none).
+    const int32_t* rnd;
+    int n_rand, nrb, nqb;
     int dk_dil[kMaxDilKinds];
     int dk_rows[kMaxDilKinds];                          // rows per TMA box for that dilation
     int dk_class_blk[kMaxDilKinds][kMaxDilTma + 1];     // block offset of class c in a head of that kind

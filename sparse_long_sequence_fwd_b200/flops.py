@@ -43,6 +43,30 @@ def row_key_counts(T: int, r: int, dil: int, globals_b=None, pad_b=None) -> np.n
     return cnt
 
 
+def rand_extra_counts(T: int, r: int, globals_b, pad_b, rb_bh) -> np.ndarray:
+    """Keys the random key blocks add to each ordinary row of one (b, h) (the
+    BigBird variant, dilation 1): the non-padded keys of the distinct blocks
+    drawn for the row's 64-row query block that lie outside the row's window
+    and are not global (int64 [T]; global rows get 0)."""
+    valid = np.ones(T, dtype=bool) if pad_b is None else ~np.asarray(pad_b, dtype=bool)
+    g = np.zeros(T, dtype=bool)
+    for x in (globals_b if globals_b is not None else []):
+        if 0 <= int(x) < T:
+            g[int(x)] = True
+    extra = np.zeros(T, dtype=np.int64)
+    rb_bh = np.asarray(rb_bh)
+    nqb = (T + 63) // 64
+    for qb in range(nqb):
+        blocks = sorted({int(c) for c in rb_bh[qb] if 0 <= int(c) < nqb})
+        for c in blocks:
+            j = np.arange(64 * c, min(64 * c + 64, T))
+            keep = valid[j] & ~g[j]
+            for i in range(64 * qb, min(64 * qb + 64, T)):
+                if not g[i]:
+                    extra[i] += int((keep & (np.abs(j - i) > r)).sum())
+    return extra
+
+
 def total_keys(B, H, T, r, dil, global_idx=None, key_pad_mask=None) -> int:
     """Sum of |N(i)| over every (b, h, i)."""
     dil = [int(x) for x in dil]

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "liblfattn.so")
 LF_F32, LF_BF16, LF_F16 = 0, 1, 2
 STATUS = {0: "LF_OK", 1: "LF_ERR_INVALID_ARG", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
           4: "LF_ERR_NO_MEMORY", 5: "LF_ERR_DEVICE_CHECK", 6: "LF_ERR_SCRATCH_TOO_SMALL"}
-EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
+EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_rand", "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
            "lf_attn_release", "lf_attn_workspace_bytes", "lf_attn_last_launch_count",
            "lf_attn_fwd_static", "lf_attn_band_plan", "lf_attn_test_hooks")
 
@@ -42,6 +42,8 @@ def load():
         sig = [P, P, P, P, I, I, I, I, I, P, P, I, P, ctypes.c_float, I, P]
         lib.lf_attn_fwd.argtypes = sig
         lib.lf_attn_fwd.restype = I
+        lib.lf_attn_fwd_rand.argtypes = sig[:15] + [P, I, P]
+        lib.lf_attn_fwd_rand.restype = I
         lib.lf_attn_fwd_stages.argtypes = sig + [ctypes.c_uint32]
         lib.lf_attn_fwd_stages.restype = I
         lib.lf_attn_fwd_host.argtypes = sig
@@ -112,10 +114,13 @@ def _check_qkv(q, k, v):
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, r: int, dil=None,
         global_idx: Optional[torch.Tensor] = None, key_pad_mask: Optional[torch.Tensor] = None,
         scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
-        stream: Optional[torch.cuda.Stream] = None, stages: int = 7) -> torch.Tensor:
+        stream: Optional[torch.cuda.Stream] = None, stages: int = 7,
+        rand_blocks: Optional[torch.Tensor] = None) -> torch.Tensor:
     """lf_attn_fwd on CUDA tensors, queued on ``stream`` (default: current stream).
 
-    ``stages`` != 7 calls lf_attn_fwd_stages (per-kernel timing)."""
+    ``stages`` != 7 calls lf_attn_fwd_stages (per-kernel timing).  ``rand_blocks``
+    (int32 [B, H, ceil(T / 64), n_rand], on the device) calls lf_attn_fwd_rand,
+    the BigBird variant."""
     _check_qkv(q, k, v)
     B, H, T, d = q.shape
     if out is None:
@@ -135,6 +140,15 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, r: int, dil=None,
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, d, int(r), _dil_array(dil, H),
             _ptr(global_idx), n_global, _ptr(key_pad_mask), float(scale), _dtype_code(q),
             ctypes.c_void_p(s.cuda_stream))
+    if rand_blocks is not None:
+        if rand_blocks.dtype != torch.int32 or not rand_blocks.is_contiguous() or rand_blocks.dim() != 4 or \
+                tuple(rand_blocks.shape[:3]) != (B, H, (T + 63) // 64) or stages != 7:
+            raise ValueError("rand_blocks must be a contiguous int32 [B, H, ceil(T / 64), n_rand] tensor")
+        n_rand = rand_blocks.shape[3]
+        st = load().lf_attn_fwd_rand(*args[:15], _ptr(rand_blocks) if n_rand else None, n_rand, args[15])
+        if st != 0:
+            raise LfAttnError(st, "lf_attn_fwd_rand")
+        return out
     if stages == 7:
         st = load().lf_attn_fwd(*args)
     else:

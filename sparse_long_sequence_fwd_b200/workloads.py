@@ -47,6 +47,7 @@ class Workload:
     pad_from: Optional[Sequence[Optional[int]]] = None  # per sample: keys >= pad_from[b] are padded
     scale: Optional[float] = None   # None -> 1/sqrt(d)
     seed: int = 0
+    n_rand: int = 0                 # BigBird variant: random key blocks per 64-row query block
 
     @property
     def softmax_scale(self) -> float:
@@ -82,7 +83,11 @@ BASE_F16 = dataclasses.replace(BASE, name="base_T4096_w513_f16", dtype="f16")
 D128 = Workload("d128_H8_T4096_w513", "bf16", 1, 8, 4096, 128, 256, _dil(8, 1),
                 globals_per_b=[[0]], scale=128 ** -0.5, seed=1006)
 
-ALL = [TINY, BASE, QA, DILATED, LARGE, BASE_F16, D128]
+# the BigBird variant of the base workload: 3 random key blocks of 64 per
+# 64-row query block (mhpn.cn page, sections 2.2.1 and 2.2.2)
+BIGBIRD = dataclasses.replace(BASE, name="bigbird_T4096_w513_rand3", n_rand=3)
+
+ALL = [TINY, BASE, QA, DILATED, LARGE, BASE_F16, D128, BIGBIRD]
 BY_NAME = {w.name: w for w in ALL}
 
 
@@ -122,10 +127,15 @@ def make_inputs(w: Workload, device: str = "cpu"):
             if p is not None:
                 pad[b, p:] = 1
 
+    rand_blocks = None
+    if w.n_rand > 0:  # drawn last, so the other inputs do not depend on it
+        nqb = (w.T + 63) // 64
+        rand_blocks = torch.randint(0, nqb, (w.B, w.H, nqb, w.n_rand), generator=g, dtype=torch.int64).to(torch.int32)
+
     out = dict(q=q, k=k, v=v, global_idx=gidx, key_pad_mask=pad,
-               dil=torch.tensor(list(w.dil), dtype=torch.int32))
+               dil=torch.tensor(list(w.dil), dtype=torch.int32), rand_blocks=rand_blocks)
     if device != "cpu":
-        for key in ("q", "k", "v", "global_idx", "key_pad_mask"):
+        for key in ("q", "k", "v", "global_idx", "key_pad_mask", "rand_blocks"):
             if out[key] is not None:
                 out[key] = out[key].to(device)
     return out
@@ -133,7 +143,7 @@ def make_inputs(w: Workload, device: str = "cpu"):
 
 def custom(name: str, dtype: str, B: int, H: int, T: int, d: int, r: int, dil=1,
            globals_per_b=None, pad_from=None, scale=None, seed: int = 7,
-           n_random_globals: int = 0) -> Workload:
+           n_random_globals: int = 0, n_rand: int = 0) -> Workload:
     """A small ad-hoc workload (edge cases in the tests)."""
     return Workload(name, dtype, B, H, T, d, r, _dil(H, dil), globals_per_b,
-                    n_random_globals, pad_from, scale, seed)
+                    n_random_globals, pad_from, scale, seed, n_rand)

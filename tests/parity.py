@@ -18,14 +18,16 @@ F32_MAX_ABS = 1e-5
 def run_gpu(w, inp, stream=None):
     dev = {k: (v.cuda() if isinstance(v, torch.Tensor) and k != "dil" else v) for k, v in inp.items()}
     out = lf_attn.fwd(dev["q"], dev["k"], dev["v"], w.r, dil=inp["dil"], global_idx=dev["global_idx"],
-                      key_pad_mask=dev["key_pad_mask"], scale=w.softmax_scale, stream=stream)
+                      key_pad_mask=dev["key_pad_mask"], scale=w.softmax_scale, stream=stream,
+                      rand_blocks=dev.get("rand_blocks"))
     torch.cuda.synchronize()
     return out
 
 
 def oracle_full(w, inp, nthreads=0):
     return oracle.fwd(inp["q"], inp["k"], inp["v"], w.r, dil=inp["dil"], global_idx=inp["global_idx"],
-                      key_pad_mask=inp["key_pad_mask"], scale=w.softmax_scale, nthreads=nthreads)
+                      key_pad_mask=inp["key_pad_mask"], scale=w.softmax_scale, nthreads=nthreads,
+                      rand_blocks=inp.get("rand_blocks"))
 
 
 def oracle_rows(w, inp, rows):

@@ -82,3 +82,21 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(lf_attn, "_lib", None)
     with pytest.raises(RuntimeError):
         lf_attn.load()
+
+
+
+def _call_rand(lib, n_rand=2, rb=P(FAKE), **kw):
+    a = dict(q=P(FAKE), k=P(FAKE), v=P(FAKE), out=P(FAKE), B=1, H=2, T=64, d=64, r=4, dil=None, g=None,
+             ng=0, pad=None, scale=0.125, dtype=1, stream=None)
+    a.update(kw)
+    return lib.lf_attn_fwd_rand(a["q"], a["k"], a["v"], a["out"], a["B"], a["H"], a["T"], a["d"], a["r"], a["dil"],
+                                a["g"], a["ng"], a["pad"], a["scale"], a["dtype"], rb, n_rand, a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_rand=5), 1), (dict(n_rand=-1), 1), (dict(rb=None), 1), (dict(n_rand=0), 1),  # table iff draws
+    (dict(rb=P(FAKE + 2)), 1),                                                          # misaligned table
+    (dict(dtype=0), 2), (dict(d=128), 2), (dict(dil=(ctypes.c_int32 * 2)(1, 2)), 2),   # bf16/f16, d 64, dil 1
+])
+def test_random_block_argument_errors(lib, kw, code):
+    assert _call_rand(lib, **kw) == code

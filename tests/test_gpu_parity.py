@@ -340,3 +340,35 @@ D128_CASES = [
 @pytest.mark.parametrize("w", D128_CASES, ids=lambda w: w.name)
 def test_d128_cases_every_element(w):
     _full_case(w)
+
+
+# The BigBird variant: window + global tokens + random key blocks of 64 per
+# 64-row query block (mhpn.cn page, sections 2.2.1 and 2.2.2), drawn by the
+# seeded input generator and passed in.
+RAND_CASES = [
+    workloads.custom("bf16_rand3", "bf16", 2, 3, 1000, 64, 60, globals_per_b=[[0, 999, 500, 500], [7, 3, 3, 640]],
+                     pad_from=[None, 777], seed=71, n_rand=3),
+    workloads.custom("f16_rand2", "f16", 1, 2, 700, 64, 20, globals_per_b=[[1, 2, 699]], seed=72, n_rand=2),
+    workloads.custom("bf16_rand1_T129", "bf16", 1, 2, 129, 64, 5, seed=73, n_rand=1),
+    workloads.custom("bf16_rand4_no_globals", "bf16", 1, 2, 600, 64, 0, seed=74, n_rand=4),
+    workloads.custom("bf16_rand3_T4096_r256", "bf16", 1, 4, 4096, 64, 256, globals_per_b=[[0]], seed=75, n_rand=3),
+    workloads.custom("bf16_rand2_40_globals", "bf16", 1, 2, 1500, 64, 30,
+                     globals_per_b=[list(range(3, 1500, 37))], pad_from=[1450], seed=76, n_rand=2),
+]
+
+
+@pytest.mark.parametrize("w", RAND_CASES, ids=lambda w: w.name)
+def test_random_blocks_every_element(w):
+    _full_case(w)
+
+
+def test_random_blocks_zero_draws_equal_plain_call():
+    w = workloads.custom("rand0", "bf16", 1, 2, 500, 64, 30, globals_per_b=[[4]], seed=77)
+    inp = workloads.make_inputs(w)
+    a = parity.run_gpu(w, inp)
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) and k != "dil" else v) for k, v in inp.items()}
+    none = torch.zeros((1, 2, 8, 0), dtype=torch.int32, device="cuda")
+    b = lf_attn.fwd(dev["q"], dev["k"], dev["v"], w.r, dil=inp["dil"], global_idx=dev["global_idx"],
+                    scale=w.softmax_scale, rand_blocks=none)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)

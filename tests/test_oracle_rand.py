@@ -136,3 +136,27 @@ def test_hand_counted_key_sets():
     assert y[129, 1] == pytest.approx((sum(range(64)) + 128 + 129) / 66, abs=1e-12)
     # row 60 (block 0, drawn block 1 is [64, 128)): its own row 60 is in the window
     assert y[60, 1] == pytest.approx((60 + sum(range(64, 128))) / 65, abs=1e-12)
+
+
+def test_flop_counter_counts_random_keys():
+    """The benchmark's key counter (flops.row_key_counts + rand_extra_counts)
+    against the brute-force membership rule above."""
+    from sparse_long_sequence_fwd_b200 import flops
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        T = int(rng.integers(1, 300))
+        r = int(rng.integers(0, 40))
+        nqb = (T + BLK - 1) // BLK
+        rb = rng.integers(-1, nqb + 1, size=(nqb, 3))
+        G = rng.integers(0, T, size=2) if rng.random() < 0.5 else None
+        pad = (rng.random(T) < 0.2) if rng.random() < 0.5 else None
+        got = flops.row_key_counts(T, r, 1, G, pad) + flops.rand_extra_counts(T, r, G, pad, rb)
+        i = np.arange(T)
+        g = np.zeros(T, dtype=bool)
+        if G is not None:
+            g[G] = True
+        allowed = (np.abs(i[:, None] - i[None, :]) <= r) | g[None, :] | g[:, None]
+        allowed |= (rb[i // BLK][:, :, None] == (i // BLK)[None, None, :]).any(axis=1)
+        if pad is not None:
+            allowed &= ~pad[None, :]
+        assert np.array_equal(got, allowed.sum(axis=1))
