@@ -139,6 +139,38 @@ lf_status lf_attn_fwd_rand(const void* q, const void* k, const void* v, void* ou
                            const int32_t* rand_blocks, int n_rand, void* stream);
 
 /*
+ * Sequence-sharded forward (several GPUs, each holding a contiguous range
+ * of the sequence; the orchestration, with its halo and global-row
+ * exchanges, is sharded.py in the Python package).  A global row attends
+ * every key ("Longformer" note, section "Global Attention"), so its softmax
+ * is split over the key shards and merged: each shard contributes the
+ * partial state (M, L, acc) of the row over its own keys, and
+ * y = sum_p 2^(M_p - M) acc_p / sum_p 2^(M_p - M) L_p with M = max_p M_p.
+ *
+ * lf_attn_rows_partial -- partial states of n_rows query rows over every
+ * non-padded key of [B, H, T, d] k and v, asynchronous on `stream`.
+ *   q_rows   DEVICE [B, H, n_rows, d], dtype `dtype` (16-byte aligned)
+ *   k, v     DEVICE [B, H, T, d] (16-byte aligned); key_pad_mask DEVICE
+ *            uint8 [B, T] or NULL
+ *   out_ml   DEVICE fp32 [B, H, n_rows, 2]: M (the largest scale * log2(e) *
+ *            q . k over the kept keys; -inf when none) and L = sum 2^(s - M)
+ *   out_acc  DEVICE fp32 [B, H, n_rows, d]: sum 2^(s - M) v
+ *   d <= 128; for LF_BF16 / LF_F16, d is 32, 64 or 128.  Uses the device
+ *   workspace of lf_attn_fwd (same rules).
+ *
+ * lf_attn_merge_rows -- merges n_parts partial states per row and writes
+ * the rows: ml [n_parts][B][H][n_rows][2], acc [n_parts][B][H][n_rows][d]
+ * (DEVICE fp32); row a of sample b goes to out row out_pos[b * n_rows + a]
+ * of the DEVICE [B, H, T_out, d] tensor `out` (dtype `dtype`), or nowhere
+ * when that entry is negative.  d <= 128.
+ */
+lf_status lf_attn_rows_partial(const void* q_rows, const void* k, const void* v, int B, int H, int n_rows,
+                               int T, int d, const uint8_t* key_pad_mask, float scale, lf_dtype dtype,
+                               float* out_ml, float* out_acc, void* stream);
+lf_status lf_attn_merge_rows(const float* ml, const float* acc, int n_parts, int B, int H, int n_rows, int d,
+                             const int32_t* out_pos, void* out, int T_out, lf_dtype dtype, void* stream);
+
+/*
  * lf_attn_fwd_stages -- runs a subset of the kernels lf_attn_fwd queues, for
  * timing one kernel at a time.  Same arguments as lf_attn_fwd, plus
  * stage_mask: bit 0 = prep (global lists, padding, packed global keys),

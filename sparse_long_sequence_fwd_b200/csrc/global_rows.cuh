@@ -141,8 +141,44 @@ __device__ __forceinline__ void stage_chunk16(float* dst, const Tin* src, int ch
     }
 }
 
-// DP: head dim rounded up to a multiple of 32 (32, 64 or 128).
-template <typename Tin, int DP>
+// Rows mode: the partial state (M, L, acc) of each of the n_rows query rows
+// over this call's keys, from the chunks' partial states (same weights as
+// merge_partials, without the division).
+__device__ __forceinline__ void merge_partials_rows(const GlobalRowParams& p, int bh, int nq, int d) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int stride = d + 2;
+    for (int a = warp; a < nq; a += kGrThreads / 32) {
+        const float* src = p.ws.partial + (static_cast<size_t>(bh) * p.gstride + a) * p.nchunk * stride;
+        float M = -INFINITY;
+        for (int c = lane; c < p.nchunk; c += 32) M = fmaxf(M, __ldcg(src + static_cast<size_t>(c) * stride));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float Mu = (M == -INFINITY) ? 0.f : M;
+        float L = 0.f;
+        for (int c = lane; c < p.nchunk; c += 32)
+            L = fmaf(exp2f(__ldcg(src + static_cast<size_t>(c) * stride) - Mu),
+                     __ldcg(src + static_cast<size_t>(c) * stride + 1), L);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        const size_t row = static_cast<size_t>(bh) * p.n_rows + a;
+        if (lane == 0) {
+            p.out_ml[2 * row] = M;
+            p.out_ml[2 * row + 1] = L;
+        }
+        for (int col = lane; col < d; col += 32) {
+            float acc = 0.f;
+            for (int c = 0; c < p.nchunk; ++c) {
+                const float* pc = src + static_cast<size_t>(c) * stride;
+                acc = fmaf(exp2f(__ldcg(pc) - Mu), __ldcg(pc + 2 + col), acc);
+            }
+            p.out_acc[row * d + col] = acc;
+        }
+    }
+}
+
+// DP: head dim rounded up to a multiple of 32 (32, 64 or 128).  kRows: rows
+// mode (GlobalRowParams).
+template <typename Tin, int DP, bool kRows = false>
 __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams p) {
     extern __shared__ __align__(16) float gr_smem[];
     float* vs = gr_smem;                  // [kChunk][DP]
@@ -157,7 +193,7 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
     const int b = bh / p.H;
     const int chunk = blockIdx.x;
     const int T = p.T, d = p.d;
-    const int nq = p.ws.n_gq[b];
+    const int nq = kRows ? p.n_rows : p.ws.n_gq[b];
     if (nq == 0) return;
 
     const Tin* kb = reinterpret_cast<const Tin*>(p.k) + static_cast<size_t>(bh) * T * d;
@@ -201,9 +237,10 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
     const int col = tid % DP, grp = tid / DP;
     const int32_t* gq = p.ws.gq_list + static_cast<size_t>(b) * p.gstride;
     for (int a = 0; a < nq; ++a) {
-        const int g = gq[a];
+        const Tin* qrow = kRows ? reinterpret_cast<const Tin*>(p.q_rows) + (static_cast<size_t>(bh) * p.n_rows + a) * d
+                                : qb + static_cast<size_t>(gq[a]) * d;
         __syncthreads();
-        if (tid < DP) qs[tid] = tid < d ? load_as_float(qb + static_cast<size_t>(g) * d + tid) : 0.f;
+        if (tid < DP) qs[tid] = tid < d ? load_as_float(qrow + tid) : 0.f;
         __syncthreads();
         float s = 0.f;
 #pragma unroll
@@ -241,8 +278,34 @@ __global__ void __launch_bounds__(kGrThreads) global_rows_kernel(GlobalRowParams
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    merge_partials<Tin>(p, bh, nq, gq, d);
+    if constexpr (kRows)
+        merge_partials_rows(p, bh, nq, d);
+    else
+        merge_partials<Tin>(p, bh, nq, gq, d);
     if (tid == 0) p.ws.counters[bh] = 0;  // ready for the next call
+}
+
+// Sequence-sharded forward: the partial states of a row from every key
+// shard combine as M = max_p M_p, w_p = 2^(M_p - M),
+// y = sum_p w_p acc_p / sum_p w_p L_p (as merge_partials does for chunks).
+// One CTA per (row a, b*h), one thread per output column.
+template <typename Tout>
+__global__ void __launch_bounds__(128) merge_rows_kernel(const __grid_constant__ MergeRowsParams p) {
+    const int a = blockIdx.x, bh = blockIdx.y, b = bh / p.H, col = threadIdx.x;
+    const int pos = p.pos[static_cast<size_t>(b) * p.n_rows + a];
+    if (pos < 0 || col >= p.d) return;
+    const size_t row = static_cast<size_t>(bh) * p.n_rows + a, per_part = static_cast<size_t>(p.BH) * p.n_rows;
+    float M = -INFINITY;
+    for (int q = 0; q < p.n_parts; ++q) M = fmaxf(M, p.ml[2 * (q * per_part + row)]);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float L = 0.f, acc = 0.f;
+    for (int q = 0; q < p.n_parts; ++q) {
+        const float w = exp2f(p.ml[2 * (q * per_part + row)] - Mu);
+        L = fmaf(w, p.ml[2 * (q * per_part + row) + 1], L);
+        acc = fmaf(w, p.acc[(q * per_part + row) * p.d + col], acc);
+    }
+    store_from_float(reinterpret_cast<Tout*>(p.out) + (static_cast<size_t>(bh) * p.T_out + pos) * p.d + col,
+                     L > 0.f ? acc / L : 0.f);
 }
 
 

@@ -169,6 +169,13 @@ lf_status set_kernel_attributes() {
                       global_rows_mma_kernel<64, true>, global_rows_mma_kernel<128, true>})
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGrSmem) != cudaSuccess)
             return LF_ERR_CUDA;
+    for (auto kern : {global_rows_kernel<float, 32, true>, global_rows_kernel<float, 64, true>,
+                      global_rows_kernel<float, 128, true>, global_rows_kernel<__nv_bfloat16, 32, true>,
+                      global_rows_kernel<__nv_bfloat16, 64, true>, global_rows_kernel<__nv_bfloat16, 128, true>,
+                      global_rows_kernel<__half, 32, true>, global_rows_kernel<__half, 64, true>,
+                      global_rows_kernel<__half, 128, true>})
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) != cudaSuccess)
+            return LF_ERR_CUDA;
     if (cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_max) != cudaSuccess ||
         cudaFuncSetAttribute(global_rows_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, gr_max) !=
             cudaSuccess ||
@@ -677,6 +684,83 @@ lf_status lf_attn_fwd_rand(const void* q, const void* k, const void* v, void* ou
     if ((st = device_state(&ds)) != LF_OK) return st;
     return launch_all(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, key_pad_mask, scale, dtype,
                       static_cast<cudaStream_t>(stream), ds, 7u, rand_blocks, n_rand);
+}
+
+lf_status lf_attn_rows_partial(const void* q_rows, const void* k, const void* v, int B, int H, int n_rows, int T,
+                               int d, const uint8_t* key_pad_mask, float scale, lf_dtype dtype, float* out_ml,
+                               float* out_acc, void* stream) {
+    if (!q_rows || !k || !v || !out_ml || !out_acc) return LF_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || n_rows < 0 || T <= 0 || d <= 0 || !std::isfinite(scale)) return LF_ERR_INVALID_ARG;
+    if (dtype != LF_F32 && dtype != LF_BF16 && dtype != LF_F16) return LF_ERR_INVALID_ARG;
+    for (const void* p : {q_rows, k, v}) if (reinterpret_cast<uintptr_t>(p) & 15u) return LF_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out_ml) | reinterpret_cast<uintptr_t>(out_acc)) & 3u) return LF_ERR_INVALID_ARG;
+    if (d > 128 || (dtype != LF_F32 && d != 32 && d != 64 && d != 128)) return LF_ERR_UNSUPPORTED;
+    if (uint64_t(B) * H > 65535u || T > kMaxT || uint64_t(B) * H * T > (uint64_t(1) << 31)) return LF_ERR_UNSUPPORTED;
+    if (n_rows == 0) return LF_OK;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    lf_status st = device_state(&ds);
+    if (st != LF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int nchunk = (T + kChunk - 1) / kChunk;
+    const size_t off_part = align256(sizeof(int32_t) * size_t(B) * H);
+    const size_t total = off_part + sizeof(float) * size_t(B) * H * n_rows * nchunk * (d + 2);
+    if ((st = grow(&ds->ws, &ds->ws_bytes, total, s)) != LF_OK) return st;
+    uint8_t* base = static_cast<uint8_t*>(ds->ws);
+    GlobalRowParams gp{};
+    gp.k = k;
+    gp.v = v;
+    gp.pad = key_pad_mask;
+    gp.ws.counters = reinterpret_cast<int32_t*>(base);
+    gp.ws.partial = reinterpret_cast<float*>(base + off_part);
+    gp.B = B; gp.H = H; gp.T = T; gp.d = d;
+    gp.gstride = n_rows;
+    gp.nchunk = nchunk;
+    gp.sl2 = static_cast<float>(double(scale) * kLog2e);
+    gp.q_rows = q_rows;
+    gp.out_ml = out_ml;
+    gp.out_acc = out_acc;
+    gp.n_rows = n_rows;
+    if (cudaMemsetAsync(gp.ws.counters, 0, sizeof(int32_t) * size_t(B) * H, s) != cudaSuccess) return LF_ERR_CUDA;
+    const dim3 grid(nchunk, B * H);
+    const int DP = d <= 32 ? 32 : (d <= 64 ? 64 : 128);
+    const size_t smem = size_t(kChunk * DP + DP + kChunk + 32 + kGrThreads) * 4;
+    void (*kern)(GlobalRowParams) =
+        dtype == LF_F32  ? (DP == 32 ? global_rows_kernel<float, 32, true>
+                            : DP == 64 ? global_rows_kernel<float, 64, true> : global_rows_kernel<float, 128, true>)
+        : dtype == LF_F16 ? (DP == 32 ? global_rows_kernel<__half, 32, true>
+                             : DP == 64 ? global_rows_kernel<__half, 64, true> : global_rows_kernel<__half, 128, true>)
+                          : (DP == 32 ? global_rows_kernel<__nv_bfloat16, 32, true>
+                             : DP == 64 ? global_rows_kernel<__nv_bfloat16, 64, true>
+                                        : global_rows_kernel<__nv_bfloat16, 128, true>);
+    kern<<<grid, kGrThreads, smem, s>>>(gp);
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+}
+
+lf_status lf_attn_merge_rows(const float* ml, const float* acc, int n_parts, int B, int H, int n_rows, int d,
+                             const int32_t* out_pos, void* out, int T_out, lf_dtype dtype, void* stream) {
+    if (!ml || !acc || !out_pos || !out) return LF_ERR_INVALID_ARG;
+    if (n_parts <= 0 || B <= 0 || H <= 0 || n_rows < 0 || d <= 0 || T_out <= 0) return LF_ERR_INVALID_ARG;
+    if (dtype != LF_F32 && dtype != LF_BF16 && dtype != LF_F16) return LF_ERR_INVALID_ARG;
+    if (d > 128 || uint64_t(B) * H > 65535u) return LF_ERR_UNSUPPORTED;
+    if (n_rows == 0) return LF_OK;
+    MergeRowsParams mp;
+    mp.ml = ml;
+    mp.acc = acc;
+    mp.pos = out_pos;
+    mp.out = out;
+    mp.n_parts = n_parts;
+    mp.BH = B * H;
+    mp.H = H;
+    mp.n_rows = n_rows;
+    mp.d = d;
+    mp.T_out = T_out;
+    const dim3 grid(n_rows, B * H);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == LF_F32) merge_rows_kernel<float><<<grid, 128, 0, s>>>(mp);
+    else if (dtype == LF_F16) merge_rows_kernel<__half><<<grid, 128, 0, s>>>(mp);
+    else merge_rows_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(mp);
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 
 lf_status lf_attn_fwd_stages(const void* q, const void* k, const void* v, void* out, int B, int H, int T, int d,

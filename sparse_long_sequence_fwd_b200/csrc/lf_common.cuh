@@ -58,6 +58,27 @@ struct GlobalRowParams {
     int cpc;                          // bf16: 128-key chunks per CTA
     int ngp;                          // bf16: rows per (b, h) of the packed global queries
     float sl2;  // scale * log2(e)
+    // Rows mode (sequence-sharded forward): the query rows come from q_rows
+    // ([B*H][n_rows][d]) instead of q at the global positions, and the merge
+    // of the chunks writes each row's partial state over these keys,
+    // out_ml [B*H][n_rows][2] = (M, L) and out_acc [B*H][n_rows][d] =
+    // sum_j 2^(s_j - M) v_j (s_j = scale * log2(e) * q . k_j), instead of y.
+    const void* q_rows;
+    float* out_ml;
+    float* out_acc;
+    int n_rows;
+};
+
+// Merge of partial row states from several key shards (sequence-sharded
+// forward): parts p = 0..n_parts-1 of ml [p][B*H][n_rows][2] and acc
+// [p][B*H][n_rows][d]; row a of sample b goes to out row pos[b][a] of
+// [B*H][T_out][d] (pos < 0: not written).
+struct MergeRowsParams {
+    const float* ml;
+    const float* acc;
+    const int32_t* pos;
+    void* out;
+    int n_parts, BH, H, n_rows, d, T_out;
 };
 
 struct BandF32Params {

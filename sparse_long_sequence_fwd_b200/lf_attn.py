@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_PKG, "liblfattn.so")
 LF_F32, LF_BF16, LF_F16 = 0, 1, 2
 STATUS = {0: "LF_OK", 1: "LF_ERR_INVALID_ARG", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
           4: "LF_ERR_NO_MEMORY", 5: "LF_ERR_DEVICE_CHECK", 6: "LF_ERR_SCRATCH_TOO_SMALL"}
-EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_rand", "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
+EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_rand", "lf_attn_rows_partial", "lf_attn_merge_rows",
+           "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
            "lf_attn_release", "lf_attn_workspace_bytes", "lf_attn_last_launch_count",
            "lf_attn_fwd_static", "lf_attn_band_plan", "lf_attn_test_hooks")
 
@@ -44,6 +45,10 @@ def load():
         lib.lf_attn_fwd.restype = I
         lib.lf_attn_fwd_rand.argtypes = sig[:15] + [P, I, P]
         lib.lf_attn_fwd_rand.restype = I
+        lib.lf_attn_rows_partial.argtypes = [P, P, P, I, I, I, I, I, P, ctypes.c_float, I, P, P, P]
+        lib.lf_attn_rows_partial.restype = I
+        lib.lf_attn_merge_rows.argtypes = [P, P, I, I, I, I, I, P, P, I, I, P]
+        lib.lf_attn_merge_rows.restype = I
         lib.lf_attn_fwd_stages.argtypes = sig + [ctypes.c_uint32]
         lib.lf_attn_fwd_stages.restype = I
         lib.lf_attn_fwd_host.argtypes = sig
@@ -155,6 +160,48 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, r: int, dil=None,
         st = load().lf_attn_fwd_stages(*args, ctypes.c_uint32(stages))
     if st != 0:
         raise LfAttnError(st, "lf_attn_fwd")
+    return out
+
+
+def rows_partial(q_rows: torch.Tensor, k: torch.Tensor, v: torch.Tensor, key_pad_mask: Optional[torch.Tensor],
+                 scale: float, stream: Optional[torch.cuda.Stream] = None):
+    """lf_attn_rows_partial: (ml fp32 [B, H, n_rows, 2], acc fp32 [B, H, n_rows, d]) of the rows
+    q_rows [B, H, n_rows, d] over the keys k, v [B, H, T, d] (CUDA tensors)."""
+    _check_qkv(k, k, v)
+    B, H, T, d = k.shape
+    if q_rows.dim() != 4 or tuple(q_rows.shape[:2]) != (B, H) or q_rows.shape[3] != d or \
+            q_rows.dtype != k.dtype or not q_rows.is_contiguous():
+        raise ValueError("q_rows must be a contiguous [B, H, n_rows, d] tensor of k's dtype")
+    n = q_rows.shape[2]
+    ml = torch.empty((B, H, n, 2), dtype=torch.float32, device=k.device)
+    acc = torch.empty((B, H, n, d), dtype=torch.float32, device=k.device)
+    if key_pad_mask is not None and (key_pad_mask.dtype != torch.uint8 or not key_pad_mask.is_contiguous()):
+        raise ValueError("key_pad_mask must be a contiguous uint8 [B, T] tensor")
+    s = stream if stream is not None else torch.cuda.current_stream(k.device)
+    st = load().lf_attn_rows_partial(_ptr(q_rows), _ptr(k), _ptr(v), B, H, n, T, d, _ptr(key_pad_mask),
+                                     float(scale), _dtype_code(k), _ptr(ml), _ptr(acc), ctypes.c_void_p(s.cuda_stream))
+    if st != 0:
+        raise LfAttnError(st, "lf_attn_rows_partial")
+    return ml, acc
+
+
+def merge_rows(ml: torch.Tensor, acc: torch.Tensor, out_pos: torch.Tensor, out: torch.Tensor,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """lf_attn_merge_rows: ml [P, B, H, n, 2], acc [P, B, H, n, d] (fp32); row a of sample b
+    goes to out[b, :, out_pos[b, a]] (skipped where out_pos < 0); out [B, H, T_out, d]."""
+    P_, B, H, n, d = acc.shape
+    if ml.shape != (P_, B, H, n, 2) or ml.dtype != torch.float32 or acc.dtype != torch.float32 or \
+            not (ml.is_contiguous() and acc.is_contiguous()):
+        raise ValueError("ml / acc must be contiguous fp32 [P, B, H, n, 2] / [P, B, H, n, d]")
+    if out_pos.shape != (B, n) or out_pos.dtype != torch.int32 or not out_pos.is_contiguous():
+        raise ValueError("out_pos must be a contiguous int32 [B, n] tensor")
+    if not out.is_contiguous() or tuple(out.shape[:2]) != (B, H) or out.shape[3] != d:
+        raise ValueError("out must be a contiguous [B, H, T_out, d] tensor")
+    s = stream if stream is not None else torch.cuda.current_stream(out.device)
+    st = load().lf_attn_merge_rows(_ptr(ml), _ptr(acc), P_, B, H, n, d, _ptr(out_pos), _ptr(out), out.shape[2],
+                                   _dtype_code(out), ctypes.c_void_p(s.cuda_stream))
+    if st != 0:
+        raise LfAttnError(st, "lf_attn_merge_rows")
     return out
 
 
