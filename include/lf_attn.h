@@ -139,6 +139,26 @@ lf_status lf_attn_fwd_rand(const void* q, const void* k, const void* v, void* ou
                            const int32_t* rand_blocks, int n_rand, void* stream);
 
 /*
+ * lf_attn_bwd -- the backward pass: gradients of the forward's output with
+ * respect to q, k and v (the pages train and fine-tune with this attention:
+ * Longformer wiki, sections 3.1 and 3.2; aiqz.cc page, gradient
+ * checkpointing), asynchronous on `stream`.  With the forward's key sets
+ * K(i), p_ij = softmax over K(i) of scale q_i . k_j, D_i = dy_i . y_i:
+ *   dv_j = sum_{i: j in K(i)} p_ij dy_i,  ds_ij = p_ij (dy_i . v_j - D_i),
+ *   dq_i = scale sum_{j in K(i)} ds_ij k_j,  dk_j = scale sum_{i: j in K(i)} ds_ij q_i.
+ *
+ *   q, k, v, y, dy  DEVICE [B,H,T,d], dtype `dtype` (y: lf_attn_fwd's output
+ *                   for these inputs; dy: the gradient of the loss w.r.t. y)
+ *   dq, dk, dv      DEVICE fp32 [B,H,T,d], fully overwritten
+ *   other arguments as lf_attn_fwd; any dtype with d <= 128 (CUDA cores).
+ *   Pointers 16-byte aligned.  Uses the device workspace of lf_attn_fwd.
+ */
+lf_status lf_attn_bwd(const void* q, const void* k, const void* v, const void* y, const void* dy,
+                      float* dq, float* dk, float* dv, int B, int H, int T, int d, int r,
+                      const int32_t* dil, const int32_t* global_idx, int n_global,
+                      const uint8_t* key_pad_mask, float scale, lf_dtype dtype, void* stream);
+
+/*
  * Sequence-sharded forward (several GPUs, each holding a contiguous range
  * of the sequence; the orchestration, with its halo and global-row
  * exchanges, is sharded.py in the Python package).  A global row attends

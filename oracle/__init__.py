@@ -186,3 +186,39 @@ def row_probs(q, k, v, r: int, b: int, h: int, i: int, dil=None, global_idx=None
 
 def max_threads() -> int:
     return int(_load().lf_oracle_max_threads())
+
+
+def bwd(q, k, v, dy, r: int, dil=None, global_idx=None, key_pad_mask=None, scale: float = None):
+    """Gradients (dq, dk, dv), fp64 numpy [B, H, T, d], of sum(y * dy) for the
+    forward's y.  Follows the forward's definition step by step in fp64 torch
+    on the CPU -- the mask view of the "Longformer" note (section "Mask
+    View": A = scale Q K^T + M, M = -inf off K(i), y = softmax(A) V) with
+    K(i) from this oracle's key_set -- and lets autograd form the gradients.
+    Rows with an empty K(i) give y = 0 and no gradient."""
+    import torch
+    qd, kd, vd, gd = (torch.from_numpy(_f32(x).astype(np.float64)) for x in (q, k, v, dy))
+    B, H, T, d = qd.shape
+    dl = _dil(dil, H)
+    gi = _i32(global_idx)
+    pad = _u8(key_pad_mask)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    qd.requires_grad_(True)
+    kd.requires_grad_(True)
+    vd.requires_grad_(True)
+    total = 0.0
+    for b in range(B):
+        G = None if gi is None else gi[b]
+        pb = None if pad is None else pad[b]
+        for h in range(H):
+            mask = torch.zeros((T, T), dtype=torch.bool)
+            for i in range(T):
+                mask[i, torch.from_numpy(key_set(T, r, int(dl[h]), i, G, pb).astype(np.int64))] = True
+            A = scale * (qd[b, h] @ kd[b, h].T)
+            A = torch.where(mask, A, torch.full_like(A, -np.inf))
+            has = mask.any(dim=1, keepdim=True)
+            P = torch.softmax(torch.where(has, A, torch.zeros_like(A)), dim=1) * has
+            y = P @ vd[b, h]
+            total = total + (y * gd[b, h]).sum()
+    total.backward()
+    return qd.grad.numpy(), kd.grad.numpy(), vd.grad.numpy()

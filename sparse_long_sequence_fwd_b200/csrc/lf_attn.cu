@@ -18,6 +18,7 @@
 #include "lf_attn.h"
 #include "band_f32.cuh"
 #include "band_tc.cuh"
+#include "bwd.cuh"
 #include "global_rows.cuh"
 #include "lf_common.cuh"
 #include "prep.cuh"
@@ -684,6 +685,88 @@ lf_status lf_attn_fwd_rand(const void* q, const void* k, const void* v, void* ou
     if ((st = device_state(&ds)) != LF_OK) return st;
     return launch_all(q, k, v, out, B, H, T, d, r, dil, global_idx, n_global, key_pad_mask, scale, dtype,
                       static_cast<cudaStream_t>(stream), ds, 7u, rand_blocks, n_rand);
+}
+
+lf_status lf_attn_bwd(const void* q, const void* k, const void* v, const void* y, const void* dy, float* dq,
+                       float* dk, float* dv, int B, int H, int T, int d, int r, const int32_t* dil,
+                       const int32_t* global_idx, int n_global, const uint8_t* key_pad_mask, float scale,
+                       lf_dtype dtype, void* stream) {
+    if (!q || !k || !v || !y || !dy || !dq || !dk || !dv) return LF_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || r < 0 || n_global < 0 || !std::isfinite(scale))
+        return LF_ERR_INVALID_ARG;
+    if ((n_global > 0) != (global_idx != nullptr)) return LF_ERR_INVALID_ARG;
+    if (dtype != LF_F32 && dtype != LF_BF16 && dtype != LF_F16) return LF_ERR_INVALID_ARG;
+    if (dil)
+        for (int h = 0; h < H; ++h)
+            if (dil[h] < 1) return LF_ERR_INVALID_ARG;
+    for (const void* p : {q, k, v, y, dy, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+        if (reinterpret_cast<uintptr_t>(p) & 15u) return LF_ERR_INVALID_ARG;
+    const uint64_t n = uint64_t(B) * uint64_t(H) * uint64_t(T) * uint64_t(d);
+    if (n / uint64_t(d) / uint64_t(T) / uint64_t(H) != uint64_t(B) || n > (uint64_t(1) << 40)) return LF_ERR_INVALID_ARG;
+    if (d > 128 || T > kMaxT || n_global > kMaxGlobal || H > kMaxHeads) return LF_ERR_UNSUPPORTED;
+    if (uint64_t(B) * H * T > (uint64_t(1) << 31) - 1) return LF_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    lf_status st = device_state(&ds);
+    if (st != LF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Layout L = make_layout(B, H, T, d, n_global, LF_F32);  // prep's lists and bitmap
+    const size_t off_stats = align256(L.total);
+    const size_t total = off_stats + sizeof(float) * 3 * size_t(B) * H * T;
+    if ((st = grow(&ds->ws, &ds->ws_bytes, total, s)) != LF_OK) return st;
+    uint8_t* base = static_cast<uint8_t*>(ds->ws);
+    Workspace ws{};
+    ws.n_gq = reinterpret_cast<int32_t*>(base + L.off_ngq);
+    ws.n_gk = reinterpret_cast<int32_t*>(base + L.off_ngk);
+    ws.gq_list = reinterpret_cast<int32_t*>(base + L.off_gq);
+    ws.gk_list = reinterpret_cast<int32_t*>(base + L.off_gk);
+    ws.gbit = reinterpret_cast<uint32_t*>(base + L.off_gbit);
+    ws.counters = reinterpret_cast<int32_t*>(base + L.off_cnt);
+    PrepParams pp{};
+    pp.gidx = global_idx;
+    pp.pad = key_pad_mask;
+    pp.q = q;
+    pp.k = k;
+    pp.v = v;
+    pp.ws = ws;
+    pp.status = ds->status;
+    pp.B = B; pp.H = H; pp.T = T; pp.d = d;
+    pp.n_global = n_global;
+    pp.gstride = L.gstride;
+    pp.ngp = L.ngp;
+    pp.W = L.W;
+    pp.pack = 0;
+    const size_t prep_smem = size_t(L.W + 2 * kPrepThreads + 2 * L.gstride) * 4;
+    prep_kernel<<<B * H, kPrepThreads, prep_smem, s>>>(pp);
+    static thread_local BwdParams bp;
+    std::memset(&bp, 0, sizeof(bp));
+    bp.q = q; bp.k = k; bp.v = v; bp.y = y; bp.dy = dy;
+    bp.dq = dq; bp.dk = dk; bp.dv = dv;
+    bp.stats = reinterpret_cast<float*>(base + off_stats);
+    bp.pad = key_pad_mask;
+    bp.ws = ws;
+    bp.B = B; bp.H = H; bp.T = T; bp.d = d; bp.r = std::min(r, T);
+    bp.gstride = L.gstride;
+    bp.W = L.W;
+    for (int h = 0; h < kMaxHeads; ++h) bp.dil[h] = (h < H && dil) ? dil[h] : 1;
+    bp.sl2 = static_cast<float>(double(scale) * kLog2e);
+    bp.scale = scale;
+    const unsigned grid = static_cast<unsigned>((uint64_t(B) * H * T + kBwdWarps - 1) / kBwdWarps);
+    if (dtype == LF_F32) {
+        bwd_stats_kernel<float><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+        bwd_dq_kernel<float><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+        bwd_dkv_kernel<float><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+    } else if (dtype == LF_F16) {
+        bwd_stats_kernel<__half><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+        bwd_dq_kernel<__half><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+        bwd_dkv_kernel<__half><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+    } else {
+        bwd_stats_kernel<__nv_bfloat16><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+        bwd_dq_kernel<__nv_bfloat16><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+        bwd_dkv_kernel<__nv_bfloat16><<<grid, kBwdWarps * 32, 0, s>>>(bp);
+    }
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 
 lf_status lf_attn_rows_partial(const void* q_rows, const void* k, const void* v, int B, int H, int n_rows, int T,

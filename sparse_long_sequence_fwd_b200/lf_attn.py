@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "liblfattn.so")
 LF_F32, LF_BF16, LF_F16 = 0, 1, 2
 STATUS = {0: "LF_OK", 1: "LF_ERR_INVALID_ARG", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
           4: "LF_ERR_NO_MEMORY", 5: "LF_ERR_DEVICE_CHECK", 6: "LF_ERR_SCRATCH_TOO_SMALL"}
-EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_rand", "lf_attn_rows_partial", "lf_attn_merge_rows",
+EXPORTS = ("lf_attn_fwd", "lf_attn_fwd_rand", "lf_attn_bwd", "lf_attn_rows_partial", "lf_attn_merge_rows",
            "lf_attn_fwd_stages", "lf_attn_fwd_host", "lf_attn_device_status", "lf_attn_strerror",
            "lf_attn_release", "lf_attn_workspace_bytes", "lf_attn_last_launch_count",
            "lf_attn_fwd_static", "lf_attn_band_plan", "lf_attn_test_hooks")
@@ -45,6 +45,8 @@ def load():
         lib.lf_attn_fwd.restype = I
         lib.lf_attn_fwd_rand.argtypes = sig[:15] + [P, I, P]
         lib.lf_attn_fwd_rand.restype = I
+        lib.lf_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, I, P, ctypes.c_float, I, P]
+        lib.lf_attn_bwd.restype = I
         lib.lf_attn_rows_partial.argtypes = [P, P, P, I, I, I, I, I, P, ctypes.c_float, I, P, P, P]
         lib.lf_attn_rows_partial.restype = I
         lib.lf_attn_merge_rows.argtypes = [P, P, I, I, I, I, I, P, P, I, I, P]
@@ -161,6 +163,31 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, r: int, dil=None,
     if st != 0:
         raise LfAttnError(st, "lf_attn_fwd")
     return out
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, y: torch.Tensor, dy: torch.Tensor, r: int, dil=None,
+        global_idx: Optional[torch.Tensor] = None, key_pad_mask: Optional[torch.Tensor] = None,
+        scale: Optional[float] = None, stream: Optional[torch.cuda.Stream] = None):
+    """lf_attn_bwd on CUDA tensors: (dq, dk, dv) fp32 [B, H, T, d] for the forward output y and
+    its gradient dy."""
+    _check_qkv(q, k, v)
+    _check_qkv(y, dy, dy)
+    if y.shape != q.shape or y.dtype != q.dtype or dy.dtype != q.dtype:
+        raise ValueError("y and dy must match q's shape and dtype")
+    B, H, T, d = q.shape
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(3))
+    n_global = 0 if global_idx is None else global_idx.shape[1]
+    if n_global == 0:
+        global_idx = None
+    if scale is None:
+        scale = d ** -0.5
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = load().lf_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), B, H, T, d,
+                            int(r), _dil_array(dil, H), _ptr(global_idx), n_global, _ptr(key_pad_mask), float(scale),
+                            _dtype_code(q), ctypes.c_void_p(s.cuda_stream))
+    if st != 0:
+        raise LfAttnError(st, "lf_attn_bwd")
+    return dq, dk, dv
 
 
 def rows_partial(q_rows: torch.Tensor, k: torch.Tensor, v: torch.Tensor, key_pad_mask: Optional[torch.Tensor],
