@@ -300,6 +300,36 @@ class WorkloadRun:
         return out
 
 
+def backward_entry(w, torch, lf_attn, dev, stream, calls=5):
+    """lf_attn_bwd on one workload: its time per call (CUDA events, after a warm-up call) and
+    useful TFLOP/s counted as 2.5x the forward's useful FLOPs (dS recomputed from Q K^T: five
+    products of 2 d FLOPs per kept (query, key) pair against the forward's two)."""
+    inp = workloads.make_inputs(w)
+    total_f = split_flops(w, inp)[0]
+    g = torch.Generator().manual_seed(w.seed + 1)
+    dy = torch.randn(inp["q"].shape, generator=g).to(inp["q"].dtype).to(dev)
+    q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
+    G = inp["global_idx"].to(dev) if inp["global_idx"] is not None else None
+    pad = inp["key_pad_mask"].to(dev) if inp["key_pad_mask"] is not None else None
+    with torch.cuda.stream(stream):
+        y = lf_attn.fwd(q, k, v, w.r, dil=inp["dil"], global_idx=G, key_pad_mask=pad, scale=w.softmax_scale,
+                        stream=stream)
+        call = lambda: lf_attn.bwd(q, k, v, y, dy, w.r, dil=inp["dil"], global_idx=G, key_pad_mask=pad,
+                                   scale=w.softmax_scale, stream=stream)
+        call()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(calls):
+            call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / calls
+    return {"value": round(2.5 * total_f / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+            "useful_gflop_per_call": round(2.5 * total_f / 1e9, 4), "calls": calls,
+            "kernels": "prep + row statistics + dq + dk/dv, CUDA cores, fp32 gradients"}
+
+
 def copy_bandwidth(torch, dev, nbytes):
     """Pinned host <-> device copy bandwidth (GB/s) for nbytes, CUDA events."""
     h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
@@ -416,6 +446,7 @@ def run_ours(args):
             others[name] = orun.summary(o_ms, peaks)
             del orun
             torch.cuda.empty_cache()
+        others["backward_" + w.name] = backward_entry(w, torch, lf_attn, dev, stream)
 
     # ---- end to end through the host-buffer entry point (pinned host memory)
     e2e = None
