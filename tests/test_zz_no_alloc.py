@@ -77,3 +77,27 @@ def test_sizes_beyond_the_scratch_are_rejected_before_launch():
     assert e.value.status == 6
     torch.cuda.synchronize()
     assert torch.all(out == 3.0)  # nothing ran
+
+
+def test_static_runs_inside_a_global_mode_graph_capture():
+    """After one call that sets the device up, lf_attn_fwd_static is captured
+    into a CUDA graph in global capture mode (where any allocation would
+    fail the capture); the replayed graph gives lf_attn_fwd's output."""
+    w = workloads.custom("static_graph", "bf16", 1, 4, 1500, 64, 60, dil=[1, 2, 1, 2],
+                         globals_per_b=[[3, 700, 1499]], pad_from=[1400], seed=52)
+    inp = workloads.make_inputs(w, "cuda")
+    kw = dict(dil=inp["dil"], global_idx=inp["global_idx"], key_pad_mask=inp["key_pad_mask"],
+              scale=w.softmax_scale)
+    ref = lf_attn.fwd(inp["q"], inp["k"], inp["v"], w.r, **kw)
+    s = torch.cuda.Stream()
+    out = torch.empty_like(inp["q"])
+    lf_attn.fwd_static(inp["q"], inp["k"], inp["v"], w.r, out=out, stream=s, **kw)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s, capture_error_mode="global"):
+        lf_attn.fwd_static(inp["q"], inp["k"], inp["v"], w.r, out=out, stream=s, **kw)
+    out.fill_(float("nan"))
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
