@@ -51,6 +51,8 @@ CASES = [
     workloads.custom("shard_bf16", "bf16", 2, 4, 2048, 64, 64, dil=[1, 2, 1, 2],
                      globals_per_b=[[0, 700, 2047, 1030], [5, 5, 1500, 1023]], pad_from=[None, 1900], seed=81),
     workloads.custom("shard_f16_d128", "f16", 1, 2, 1500, 128, 100, globals_per_b=[[0, 760]], seed=82),
+    workloads.custom("shard_f32", "f32", 1, 2, 800, 64, 40, dil=[1, 2], globals_per_b=[[10, 500]], pad_from=[790],
+                     seed=83),
 ]
 
 
