@@ -69,6 +69,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int kMaxBandCtas = 296;
 // ... for a head dimension (one CTA per SM at HD = 128)
 constexpr int max_band_ctas(int d) { return d == 64 ? kMaxBandCtas : kMaxBandCtas / 2; }
+constexpr int kFewGlobals = 4;        // global tokens up to which ...
+constexpr int kFewGlobalsSlots = 24;  // ... the band kernel leaves this many CTA slots free
 
 struct Layout {
     size_t off_ngq, off_ngk, off_gq, off_gk, off_gbit, off_cnt, off_part, off_kg, off_vg, off_qg, off_bcnt, off_bpart,
@@ -492,10 +494,15 @@ lf_status launch_all(const void* q, const void* k, const void* v, void* out, int
         bp.n_rand = n_rand;
         bp.nrb = nrb;
         bp.nqb = (T + kBN - 1) / kBN;
+        // With a few global rows (their stage is short), some SM slots are left to the
+        // global-row kernel from the start instead of only in the band kernel's tail.  (The
+        // same launch shape whichever stages or entry point run, so a band-only call times
+        // the same kernel and every entry point gives the same bits.)
+        int band_ctas = std::min((d == 64 ? BandCfg<64>::kCtasPerSm : BandCfg<128>::kCtasPerSm) * ds->sm_count,
+                                 max_band_ctas(d));
+        if (d == 64 && n_global > 0 && n_global <= kFewGlobals) band_ctas -= kFewGlobalsSlots;
         if ((st = band_schedule(bp, B, H, T, r_eff, nrb + (n_global > 0 ? (L.gstride + kBN - 1) / kBN : 0), kind_of_head,
-                                std::min((d == 64 ? BandCfg<64>::kCtasPerSm : BandCfg<128>::kCtasPerSm) * ds->sm_count,
-                                         max_band_ctas(d)),
-                                L.band_tiles)) != LF_OK)
+                                band_ctas, L.band_tiles)) != LF_OK)
             return st;
         bp.cnt = reinterpret_cast<int32_t*>(base + L.off_bcnt);
         bp.part = reinterpret_cast<float*>(base + L.off_bpart);
