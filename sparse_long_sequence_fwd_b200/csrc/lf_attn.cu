@@ -90,10 +90,13 @@ Layout make_layout(int B, int H, int T, int d, int n_global, lf_dtype dtype) {
         const int nblk = (T + kGrKeys - 1) / kGrKeys;
         // Warps split each chunk's keys when there are few global queries, but
         // combining the slices only pays off when a CTA takes two chunks or more.
+        // With few global tokens the band kernel leaves CTA slots free (launch_all),
+        // and fewer, longer global-row CTAs (about two per SM) finish sooner in them.
+        const long budget = n_global <= kFewGlobals ? 296 : 444;
         auto chunks_per_cta = [&](int kpw) {
             const int rows = kpw / 2;  // global-query slots per CTA
             const long units = long(nblk) * B * H * ((L.gstride + rows - 1) / rows);
-            return static_cast<int>(std::max(1L, std::min<long>(nblk, (units + 443) / 444)));
+            return static_cast<int>(std::max(1L, std::min<long>(nblk, (units + budget - 1) / budget)));
         };
         L.gr_kpw = gr_kpw(L.gstride);
         L.cpc = chunks_per_cta(L.gr_kpw);
