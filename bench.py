@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only lf_attn_bwd on --workload and print that entry (for profiling the backward)")
     ap.add_argument("--no-others", action="store_true",
                     help="skip the QA, dilated, large, f16 base, d = 128 and BigBird workload entries")
     return ap.parse_args()
@@ -374,6 +376,9 @@ def run_ours(args):
     stream = torch.cuda.Stream(device=dev)
 
     w = workloads.BY_NAME[args.workload]
+    if args.backward_only:
+        print(json.dumps({"backward_" + w.name: backward_entry(w, torch, lf_attn, dev, stream)}))
+        return
     run = WorkloadRun(w, torch, lf_attn, dev, stream, args.warmup)
     launches_per_step = run.launches_per_step
     K = args.steps
